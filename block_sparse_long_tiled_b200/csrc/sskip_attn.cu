@@ -1,0 +1,308 @@
+// sskip_attn.cu -- the C ABI of libsskip_attn.so (declared in
+// include/sskip_attn.h): argument validation, TMA descriptor set-up and the
+// launches of the sm_100a kernels.  One translation unit, so the device status
+// word is shared by every kernel without relocatable device code.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/sskip_attn.h"
+#include "decode_sm100.cuh"
+#include "prefill_sm100.cuh"
+
+#define SSKIP_API extern "C" __attribute__((visibility("default")))
+
+namespace sskip {
+
+// A kernel that waits on an mbarrier nothing will ever complete: its bounded
+// wait must run out, latch SSKIP_ERR_TIMEOUT and return.
+__global__ void watchdog_selftest_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, (volatile int*)&abort_flag, limit_ns);
+}
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 map over a [planes, rows, d] tensor, box {64, box_rows, 1},
+// 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* map, const void* base, int d, int rows, long long planes, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)planes};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * (cuuint64_t)rows};
+  cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev;
+}
+
+// Raise a kernel's dynamic shared memory limit once per device.
+template <typename K>
+cudaError_t ensure_smem(K kernel, int bytes) {
+  static std::mutex mu;
+  static unsigned long long done_mask = 0;  // one bit per device (first 64)
+  const int dev = current_device();
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev < 64 && (done_mask >> dev) & 1ull) return cudaSuccess;
+  }
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev < 64) {
+    std::lock_guard<std::mutex> lk(mu);
+    done_mask |= 1ull << dev;
+  }
+  return e;
+}
+
+template <int D, int BR, int BC, bool CAUSAL>
+int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                   const PrefillParams& p, cudaStream_t st) {
+  auto kernel = prefill_kernel<D, BR, BC, CAUSAL>;
+  const int smem = PrefillCfg<D, BC>::kAlloc;
+  if (ensure_smem(kernel, smem) != cudaSuccess) return SSKIP_ERR_CUDA;
+  const long long grid = (long long)p.B * p.Hq * p.n_units;
+  kernel<<<(unsigned)grid, kPfThreads, smem, st>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? SSKIP_OK : SSKIP_ERR_CUDA;
+}
+
+template <int D, int G>
+int launch_decode(const DecodeParams& p, cudaStream_t st) {
+  auto kernel = decode_split_kernel<D, G>;
+  const int smem = DecodeSmem<D, G>::kTotal;
+  if (ensure_smem(kernel, smem) != cudaSuccess) return SSKIP_ERR_CUDA;
+  dim3 grid(p.S, p.Hkv, p.B);
+  kernel<<<grid, kDecThreads, smem, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return SSKIP_ERR_CUDA;
+  decode_combine_kernel<D><<<(unsigned)(p.B * p.Hq), 128, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SSKIP_OK : SSKIP_ERR_CUDA;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+}  // namespace sskip
+
+using namespace sskip;
+
+SSKIP_API int sskip_version(void) { return kVersion; }
+
+SSKIP_API const char* sskip_status_string(int status) {
+  switch (status) {
+    case SSKIP_OK: return "ok";
+    case SSKIP_ERR_INVALID_ARG: return "invalid argument";
+    case SSKIP_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SSKIP_ERR_CUDA: return "CUDA error";
+    case SSKIP_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+SSKIP_API int sskip_device_supported(int device) {
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return SSKIP_ERR_CUDA;
+  return (prop.major == 10 && prop.minor == 0) ? SSKIP_OK : SSKIP_ERR_UNSUPPORTED;
+}
+
+SSKIP_API int sskip_attn_prefill_ex(const void* q, const void* k, const void* v, void* o,
+                                    float* lse, int B, int Hq, int Hkv, int L, int d, int causal,
+                                    float sm_scale, float threshold_scale_factor, int Br, int Bc,
+                                    unsigned long long* skip_count, uint8_t* tile_state,
+                                    void* stream) {
+  if (!q || !k || !v || !o || !lse) return SSKIP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(skip_count) & 7u))
+    return SSKIP_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0) return SSKIP_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SSKIP_ERR_INVALID_ARG;
+  if (!(threshold_scale_factor >= 0.f) || !std::isfinite(threshold_scale_factor))
+    return SSKIP_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SSKIP_ERR_UNSUPPORTED;
+  if (!((Br == 64 && Bc == 64) || (Br == 128 && Bc == 128))) return SSKIP_ERR_UNSUPPORTED;
+  const long long n_units = (L + 127) / 128;
+  if ((long long)B * Hq * n_units >= (1ll << 31) || (long long)B * Hq >= (1ll << 31))
+    return SSKIP_ERR_UNSUPPORTED;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, d, L, (long long)B * Hq, 128) ||
+      !make_map(&mk, k, d, L, (long long)B * Hkv, Bc) ||
+      !make_map(&mv, v, d, L, (long long)B * Hkv, Bc))
+    return SSKIP_ERR_CUDA;
+
+  PrefillParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.counts = skip_count;
+  p.tile_state = tile_state;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.G = Hq / Hkv;
+  p.n_q = (L + Br - 1) / Br;
+  p.n_k = (L + Bc - 1) / Bc;
+  p.n_units = (int)n_units;
+  p.scale_log2 = (float)((double)sm_scale * 1.4426950408889634);
+  p.t_positive = threshold_scale_factor > 0.f;
+  p.log2_t = p.t_positive ? (float)std::log2((double)threshold_scale_factor / (double)L)
+                          : -INFINITY;
+
+  if (skip_count && cudaMemsetAsync(skip_count, 0, 2 * sizeof(unsigned long long), st) != cudaSuccess)
+    return SSKIP_ERR_CUDA;
+  if (tile_state &&
+      cudaMemsetAsync(tile_state, 0, (size_t)B * Hq * p.n_q * p.n_k, st) != cudaSuccess)
+    return SSKIP_ERR_CUDA;
+
+  const bool c = causal != 0;
+  if (d == 128 && Br == 128) return c ? launch_prefill<128, 128, 128, true>(mq, mk, mv, p, st)
+                                      : launch_prefill<128, 128, 128, false>(mq, mk, mv, p, st);
+  if (d == 64 && Br == 128) return c ? launch_prefill<64, 128, 128, true>(mq, mk, mv, p, st)
+                                     : launch_prefill<64, 128, 128, false>(mq, mk, mv, p, st);
+  if (d == 128 && Br == 64) return c ? launch_prefill<128, 64, 64, true>(mq, mk, mv, p, st)
+                                     : launch_prefill<128, 64, 64, false>(mq, mk, mv, p, st);
+  return c ? launch_prefill<64, 64, 64, true>(mq, mk, mv, p, st)
+           : launch_prefill<64, 64, 64, false>(mq, mk, mv, p, st);
+}
+
+SSKIP_API int sskip_attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 int B, int Hq, int Hkv, int L, int d, int causal, float sm_scale,
+                                 float threshold_scale_factor, int Br, int Bc,
+                                 unsigned long long* skip_count, void* stream) {
+  return sskip_attn_prefill_ex(q, k, v, o, lse, B, Hq, Hkv, L, d, causal, sm_scale,
+                               threshold_scale_factor, Br, Bc, skip_count, nullptr, stream);
+}
+
+SSKIP_API size_t sskip_attn_decode_workspace_size(int B, int Hq, int d, int num_splits) {
+  if (B < 1 || Hq < 1 || d < 1 || num_splits < 1) return 0;
+  const size_t rows = (size_t)B * Hq * num_splits;
+  return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+SSKIP_API int sskip_attn_decode_ex(const void* q, const void* kcache, const void* vcache,
+                                   const int* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
+                                   int Lmax, int d, float sm_scale, float threshold_scale_factor,
+                                   int Bc, int num_splits, void* workspace, size_t workspace_bytes,
+                                   unsigned long long* skip_count, uint8_t* tile_state,
+                                   void* stream) {
+  if (!q || !kcache || !vcache || !seqlens || !o || !lse || !workspace)
+    return SSKIP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(skip_count) & 7u))
+    return SSKIP_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lmax < 1 || Hq % Hkv != 0 || num_splits < 1)
+    return SSKIP_ERR_INVALID_ARG;
+  if (B > 65535 || Hkv > 65535) return SSKIP_ERR_UNSUPPORTED;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SSKIP_ERR_INVALID_ARG;
+  if (!(threshold_scale_factor >= 0.f) || !std::isfinite(threshold_scale_factor))
+    return SSKIP_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (d != 64 && d != 128) return SSKIP_ERR_UNSUPPORTED;
+  if (Bc != kDecBc || num_splits > 64) return SSKIP_ERR_UNSUPPORTED;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return SSKIP_ERR_UNSUPPORTED;
+  if (workspace_bytes < sskip_attn_decode_workspace_size(B, Hq, d, num_splits))
+    return SSKIP_ERR_INVALID_ARG;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t rows = (size_t)B * Hq * num_splits;
+  DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kc = static_cast<const __nv_bfloat16*>(kcache);
+  p.vc = static_cast<const __nv_bfloat16*>(vcache);
+  p.seqlens = seqlens;
+  p.o_part = static_cast<float*>(workspace);
+  p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * d * 4));
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.counts = skip_count;
+  p.tile_state = tile_state;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lmax = Lmax; p.S = num_splits;
+  p.n_k_max = (Lmax + kDecBc - 1) / kDecBc;
+  p.scale_log2 = (float)((double)sm_scale * 1.4426950408889634);
+  p.tsf = threshold_scale_factor;
+
+  if (skip_count && cudaMemsetAsync(skip_count, 0, 2 * sizeof(unsigned long long), st) != cudaSuccess)
+    return SSKIP_ERR_CUDA;
+  if (tile_state &&
+      cudaMemsetAsync(tile_state, 0, (size_t)B * Hkv * p.n_k_max, st) != cudaSuccess)
+    return SSKIP_ERR_CUDA;
+
+  if (d == 128) {
+    switch (G) {
+      case 1: return launch_decode<128, 1>(p, st);
+      case 2: return launch_decode<128, 2>(p, st);
+      case 4: return launch_decode<128, 4>(p, st);
+      default: return launch_decode<128, 8>(p, st);
+    }
+  }
+  switch (G) {
+    case 1: return launch_decode<64, 1>(p, st);
+    case 2: return launch_decode<64, 2>(p, st);
+    case 4: return launch_decode<64, 4>(p, st);
+    default: return launch_decode<64, 8>(p, st);
+  }
+}
+
+SSKIP_API int sskip_attn_decode(const void* q, const void* kcache, const void* vcache,
+                                const int* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
+                                int Lmax, int d, float sm_scale, float threshold_scale_factor,
+                                int Bc, int num_splits, void* workspace, size_t workspace_bytes,
+                                unsigned long long* skip_count, void* stream) {
+  return sskip_attn_decode_ex(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Lmax, d, sm_scale,
+                              threshold_scale_factor, Bc, num_splits, workspace, workspace_bytes,
+                              skip_count, nullptr, stream);
+}
+
+SSKIP_API int sskip_get_status(void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SSKIP_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return SSKIP_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return SSKIP_ERR_CUDA;
+  }
+  return v;
+}
+
+SSKIP_API int sskip_selftest_watchdog(unsigned int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 2000000u) return SSKIP_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  watchdog_selftest_kernel<<<1, 32, 0, st>>>((uint64_t)limit_us * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? SSKIP_OK : SSKIP_ERR_CUDA;
+}

@@ -1,0 +1,168 @@
+/*
+ * sskip_attn.h -- C ABI of libsskip_attn.so: Skip-Softmax tiled attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * What the library computes
+ * -------------------------
+ * FlashAttention-style tiled attention in which a block of logits is skipped
+ * when it sits far enough below the running maximum.  The TensorRT-LLM
+ * Skip-Softmax article ("TRT-LLM sparse attention, 1.4x", section
+ * "Skip Softmax 的三步走算法") gives the test in three steps: take the block's
+ * local maximum logit; compare it with the running global maximum; when the
+ * gap exceeds the threshold, skip the block's softmax, its second matmul
+ * (P.V) and the load of its V block from HBM.  The same article ("实战演练"
+ * section) defines the threshold as threshold_scale_factor divided by the
+ * context length: t = threshold_scale_factor / L.
+ *
+ * Exactly:  for query-tile rows r and key tile j (visited in ascending j),
+ *   m_local[r] = max over visible keys of sm_scale * q_r . k_c
+ *   row r passes  iff  m_local[r] - m_run[r] < ln t     (strict; ln 0 = -inf)
+ *   the tile is skipped iff every valid row passes; a skipped tile changes
+ *   neither the running max m, nor the row sum l, nor the accumulator O;
+ *   a kept tile runs the usual online-softmax update and O += P V.
+ * The first visited tile of every row is never skipped (m_run = -inf).
+ * threshold_scale_factor = 0 reproduces dense softmax attention.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device, owned
+ *    by the caller, 16-byte aligned, densely packed in the layouts stated.
+ *    bf16 tensors are raw IEEE bfloat16 (uint16 storage).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call is asynchronous on that stream and allocates nothing.
+ *  - The return value reports argument validation and launch errors
+ *    synchronously (sskip_status).  Errors found on the device while a kernel
+ *    runs (a bounded wait that ran out) are latched in a per-device status
+ *    word that sskip_get_status() reads.  No C++ exception crosses this ABI.
+ *  - Outputs, the counters included, are overwritten, never accumulated.
+ */
+#ifndef SSKIP_ATTN_H_
+#define SSKIP_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSKIP_OK = 0,
+    SSKIP_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, misaligned, tsf < 0 */
+    SSKIP_ERR_UNSUPPORTED = 2,  /* valid but not built: d, tile sizes, device  */
+    SSKIP_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed        */
+    SSKIP_ERR_TIMEOUT = 4       /* a bounded device-side wait ran out          */
+} sskip_status;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int sskip_version(void);
+
+/* Human-readable name of a status code (static string; never NULL). */
+const char* sskip_status_string(int status);
+
+/* Returns SSKIP_OK when `device` is an sm_100 GPU this build runs on,
+ * SSKIP_ERR_UNSUPPORTED otherwise, SSKIP_ERR_CUDA if the query failed. */
+int sskip_device_supported(int device);
+
+/*
+ * Prefill: causal or non-causal Skip-Softmax attention over one sequence per
+ * batch entry (the compute-bound phase of the article's "Skip Softmax 带来了
+ * 哪些实战好处" section: skipping the softmax and BMM2 removes FLOPs).
+ *
+ *   q   [B, Hq,  L, d] bf16      o   [B, Hq, L, d] bf16 (written)
+ *   k   [B, Hkv, L, d] bf16      lse [B, Hq, L] fp32, natural log of the
+ *   v   [B, Hkv, L, d] bf16          row sum over the KEPT keys (written)
+ *
+ *   Query head hq reads kv head hq / (Hq / Hkv) (grouped-query attention).
+ *   causal: key c is visible to row r iff c <= r.  Tiles wholly above the
+ *   diagonal are not visited and not counted.
+ *   sm_scale: logit scale (commonly 1/sqrt(d)).
+ *   threshold_scale_factor >= 0: t = threshold_scale_factor / L.
+ *   Br, Bc: query / key tile sizes; the skip decision is taken per Br x Bc
+ *   tile of ONE query head.  Supported: (Br, Bc) in {(64, 64), (128, 128)}.
+ *   d in {64, 128}.  L >= 1, Hq % Hkv == 0.
+ *   skip_count: optional device uint64[2] = {skipped tiles, visited tiles}
+ *   summed over the call; may be NULL.
+ */
+int sskip_attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
+                       int B, int Hq, int Hkv, int L, int d, int causal, float sm_scale,
+                       float threshold_scale_factor, int Br, int Bc,
+                       unsigned long long* skip_count, void* stream);
+
+/*
+ * Same as sskip_attn_prefill, plus an optional per-tile record of the
+ * decisions: tile_state [B, Hq, ceil(L/Br), ceil(L/Bc)] uint8 on the device,
+ * 0 = not visited, 1 = kept, 2 = skipped.  NULL disables it.
+ */
+int sskip_attn_prefill_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Hq, int Hkv, int L, int d, int causal, float sm_scale,
+                          float threshold_scale_factor, int Br, int Bc,
+                          unsigned long long* skip_count, uint8_t* tile_state, void* stream);
+
+/*
+ * Decode: one new query token per sequence against a contiguous KV cache,
+ * split over the key axis and merged by log-sum-exp (the bandwidth-bound
+ * phase of the article's "Skip Softmax 带来了哪些实战好处" section: a skipped
+ * block costs no V load).
+ *
+ *   q       [B, Hq, d] bf16               o   [B, Hq, d] bf16 (written)
+ *   kcache  [B, Hkv, Lmax, d] bf16         lse [B, Hq] fp32 natural log
+ *   vcache  [B, Hkv, Lmax, d] bf16             (written)
+ *   seqlens [B] int32 on the device, 1 <= seqlens[b] <= Lmax; rows at or
+ *           beyond seqlens[b] are never read.
+ *
+ *   A decode tile is the G = Hq / Hkv query heads that share one kv head
+ *   times Bc keys; the G heads take ONE joint decision, so a skipped tile
+ *   really loads no V bytes.  t_b = threshold_scale_factor / seqlens[b].
+ *   The key tiles of each (b, kv head) are cut into num_splits contiguous
+ *   chunks of c = ceil(n_k / num_splits) tiles (n_k = ceil(seqlens[b] / Bc));
+ *   each chunk runs its own online softmax from m_run = -inf, and the chunks
+ *   merge by log-sum-exp.
+ *   Supported: d in {64, 128}, Bc = 64, G in {1, 2, 4, 8}, 1 <= num_splits <= 64.
+ *   workspace: device scratch of at least
+ *   sskip_attn_decode_workspace_size(B, Hq, d, num_splits) bytes, 256-byte
+ *   aligned, owned by the caller; its contents need no initialisation and
+ *   are meaningless after the call.
+ *   skip_count: optional device uint64[2] = {skipped, visited} decode tiles.
+ */
+size_t sskip_attn_decode_workspace_size(int B, int Hq, int d, int num_splits);
+
+int sskip_attn_decode(const void* q, const void* kcache, const void* vcache,
+                      const int* seqlens, void* o, float* lse,
+                      int B, int Hq, int Hkv, int Lmax, int d, float sm_scale,
+                      float threshold_scale_factor, int Bc, int num_splits,
+                      void* workspace, size_t workspace_bytes,
+                      unsigned long long* skip_count, void* stream);
+
+/* Same as sskip_attn_decode, plus tile_state [B, Hkv, ceil(Lmax/Bc)] uint8
+ * (0 = not visited, 1 = kept, 2 = skipped); NULL disables it. */
+int sskip_attn_decode_ex(const void* q, const void* kcache, const void* vcache,
+                         const int* seqlens, void* o, float* lse,
+                         int B, int Hq, int Hkv, int Lmax, int d, float sm_scale,
+                         float threshold_scale_factor, int Bc, int num_splits,
+                         void* workspace, size_t workspace_bytes,
+                         unsigned long long* skip_count, uint8_t* tile_state, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's status
+ * word: SSKIP_OK, or the first device-side error latched since the last call
+ * (SSKIP_ERR_TIMEOUT when a bounded wait inside a kernel ran out; the kernel
+ * then abandoned its work and its outputs are undefined).  Returns
+ * SSKIP_ERR_CUDA if the synchronisation itself failed.
+ */
+int sskip_get_status(void* stream);
+
+/*
+ * Self-test of the bounded-wait watchdog: launches one tiny kernel that waits
+ * on an mbarrier that nothing ever completes, with a wait limit of
+ * `limit_us` microseconds (1 .. 2,000,000).  The wait runs out, the kernel
+ * latches SSKIP_ERR_TIMEOUT in the status word and returns; the context stays
+ * usable.  Read the result with sskip_get_status().
+ */
+int sskip_selftest_watchdog(unsigned int limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSKIP_ATTN_H_ */

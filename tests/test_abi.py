@@ -1,0 +1,110 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/sskip_attn.h declares, and rejects bad arguments before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_long_tiled_b200 as sk
+from block_sparse_long_tiled_b200 import build as sk_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sskip_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sk_build.build()
+    return sk.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(sskip_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_expected_api():
+    names = header_functions()
+    assert "sskip_attn_prefill" in names and "sskip_attn_decode" in names
+    assert set(names) == set(sk.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+    assert lib.sskip_version() == 100
+
+
+def test_status_strings(lib):
+    assert sk.status_string(0) == "ok"
+    assert "timed out" in sk.status_string(4)
+    assert sk.status_string(99) == "unknown status"
+
+
+def test_decode_workspace_size(lib):
+    B, Hq, d, S = 64, 32, 128, 16
+    rows = B * Hq * S
+    want = ((rows * d * 4 + 255) // 256) * 256 + ((rows * 4 + 255) // 256) * 256
+    assert sk.sskip_attn_decode_workspace_size(B, Hq, d, S) == want
+    assert sk.sskip_attn_decode_workspace_size(0, Hq, d, S) == 0
+
+
+FAKE = ctypes.c_void_p(1 << 20)      # 16-byte aligned, never dereferenced
+FAKE_ODD = ctypes.c_void_p((1 << 20) + 8)
+
+
+def prefill_call(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=1, L=128, d=128,
+                 causal=1, scale=0.088, tsf=10.0, Br=128, Bc=128, counts=None):
+    return lib.sskip_attn_prefill(q, k, v, o, lse, B, Hq, Hkv, L, d, causal, scale, tsf, Br, Bc,
+                                  counts, None)
+
+
+def test_prefill_argument_validation(lib):
+    assert prefill_call(lib, q=None) == sk.SSKIP_ERR_INVALID_ARG
+    assert prefill_call(lib, k=FAKE_ODD) == sk.SSKIP_ERR_INVALID_ARG
+    assert prefill_call(lib, L=0) == sk.SSKIP_ERR_INVALID_ARG
+    assert prefill_call(lib, Hq=3, Hkv=2) == sk.SSKIP_ERR_INVALID_ARG
+    assert prefill_call(lib, tsf=-1.0) == sk.SSKIP_ERR_INVALID_ARG
+    assert prefill_call(lib, tsf=float("inf")) == sk.SSKIP_ERR_INVALID_ARG
+    assert prefill_call(lib, scale=0.0) == sk.SSKIP_ERR_INVALID_ARG
+    assert prefill_call(lib, d=96) == sk.SSKIP_ERR_UNSUPPORTED
+    assert prefill_call(lib, Br=64, Bc=128) == sk.SSKIP_ERR_UNSUPPORTED
+    assert prefill_call(lib, counts=ctypes.c_void_p((1 << 20) + 4)) == sk.SSKIP_ERR_INVALID_ARG
+
+
+def decode_call(lib, q=FAKE, ws=FAKE, ws_bytes=1 << 30, B=2, Hq=8, Hkv=2, Lmax=256, d=128,
+                Bc=64, S=4, tsf=5.0, seqlens=FAKE):
+    return lib.sskip_attn_decode(q, FAKE, FAKE, seqlens, FAKE, FAKE, B, Hq, Hkv, Lmax, d, 0.088,
+                                 tsf, Bc, S, ws, ws_bytes, None, None)
+
+
+def test_decode_argument_validation(lib):
+    assert decode_call(lib, q=None) == sk.SSKIP_ERR_INVALID_ARG
+    assert decode_call(lib, ws=None) == sk.SSKIP_ERR_INVALID_ARG
+    assert decode_call(lib, ws=ctypes.c_void_p((1 << 20) + 16)) == sk.SSKIP_ERR_INVALID_ARG
+    assert decode_call(lib, ws_bytes=16) == sk.SSKIP_ERR_INVALID_ARG
+    assert decode_call(lib, Hq=6, Hkv=4) == sk.SSKIP_ERR_INVALID_ARG
+    assert decode_call(lib, tsf=-2.0) == sk.SSKIP_ERR_INVALID_ARG
+    assert decode_call(lib, Bc=128) == sk.SSKIP_ERR_UNSUPPORTED
+    assert decode_call(lib, Hq=24, Hkv=2) == sk.SSKIP_ERR_UNSUPPORTED   # G = 12
+    assert decode_call(lib, S=65) == sk.SSKIP_ERR_UNSUPPORTED
+    assert decode_call(lib, d=32) == sk.SSKIP_ERR_UNSUPPORTED
+
+
+def test_watchdog_selftest_rejects_bad_limits(lib):
+    assert lib.sskip_selftest_watchdog(0, None) == sk.SSKIP_ERR_INVALID_ARG
+    assert lib.sskip_selftest_watchdog(3_000_000, None) == sk.SSKIP_ERR_INVALID_ARG
+
+
+def test_product_path_has_no_oracle_dependency():
+    # The CUDA binding and its sources never reach the CPU oracle.
+    pkg = os.path.join(ROOT, "block_sparse_long_tiled_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src, f
+                assert "sskip_oracle" not in src, f
