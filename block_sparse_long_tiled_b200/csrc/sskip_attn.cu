@@ -10,6 +10,8 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "../../include/sskip_attn.h"
 #include "decode_sm100.cuh"
@@ -74,21 +76,15 @@ int current_device() {
   return dev;
 }
 
-// Raise a kernel's dynamic shared memory limit once per device.
-template <typename K>
-cudaError_t ensure_smem(K kernel, int bytes) {
+// Raise a kernel's dynamic shared memory limit once per (kernel, device).
+cudaError_t ensure_smem(const void* kernel, int bytes) {
   static std::mutex mu;
-  static unsigned long long done_mask = 0;  // one bit per device (first 64)
-  const int dev = current_device();
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    if (dev < 64 && (done_mask >> dev) & 1ull) return cudaSuccess;
-  }
+  static std::set<std::pair<const void*, int>> done;
+  const std::pair<const void*, int> key(kernel, current_device());
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.count(key)) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && dev < 64) {
-    std::lock_guard<std::mutex> lk(mu);
-    done_mask |= 1ull << dev;
-  }
+  if (e == cudaSuccess) done.insert(key);
   return e;
 }
 
@@ -97,7 +93,8 @@ int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorM
                    const PrefillParams& p, cudaStream_t st) {
   auto kernel = prefill_kernel<D, BR, BC, CAUSAL>;
   const int smem = PrefillCfg<D, BC>::kAlloc;
-  if (ensure_smem(kernel, smem) != cudaSuccess) return SSKIP_ERR_CUDA;
+  if (ensure_smem(reinterpret_cast<const void*>(kernel), smem) != cudaSuccess)
+    return SSKIP_ERR_CUDA;
   const long long grid = (long long)p.B * p.Hq * p.n_units;
   kernel<<<(unsigned)grid, kPfThreads, smem, st>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? SSKIP_OK : SSKIP_ERR_CUDA;
@@ -107,7 +104,8 @@ template <int D, int G>
 int launch_decode(const DecodeParams& p, cudaStream_t st) {
   auto kernel = decode_split_kernel<D, G>;
   const int smem = DecodeSmem<D, G>::kTotal;
-  if (ensure_smem(kernel, smem) != cudaSuccess) return SSKIP_ERR_CUDA;
+  if (ensure_smem(reinterpret_cast<const void*>(kernel), smem) != cudaSuccess)
+    return SSKIP_ERR_CUDA;
   dim3 grid(p.S, p.Hkv, p.B);
   kernel<<<grid, kDecThreads, smem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return SSKIP_ERR_CUDA;
