@@ -81,13 +81,20 @@ def load_peaks() -> tuple[dict, str]:
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "prefill_kernel": ("prefill_sm100.cuh", "sm100_ptx.cuh", "skip_rule.cuh"),
+    "decode_split_kernel": ("decode_sm100.cuh", "sm100_ptx.cuh", "skip_rule.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the sources one kernel is compiled from (its ncu record is
+    stale as soon as they change)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_long_tiled_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -99,7 +106,7 @@ def ncu_traffic(kernel: str) -> float | None:
         return None
     with open(path) as f:
         rec = json.load(f).get(kernel)
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or rec.get("source_hash") != kernel_source_hash(kernel):
         return None
     return float(rec["dram_bytes_per_launch"])
 
