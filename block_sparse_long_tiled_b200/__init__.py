@@ -25,8 +25,11 @@ SSKIP_OK, SSKIP_ERR_INVALID_ARG, SSKIP_ERR_UNSUPPORTED, SSKIP_ERR_CUDA, SSKIP_ER
 
 EXPORTS = ("sskip_version", "sskip_status_string", "sskip_device_supported",
            "sskip_attn_prefill", "sskip_attn_prefill_ex", "sskip_attn_decode_workspace_size",
-           "sskip_attn_decode", "sskip_attn_decode_ex", "sskip_get_status",
-           "sskip_selftest_watchdog")
+           "sskip_attn_decode", "sskip_attn_decode_ex", "sskip_attn_decode_noalloc",
+           "sskip_get_status", "sskip_selftest_watchdog")
+
+# Size of the library's fixed decode scratch (see sskip_attn_decode_noalloc).
+DECODE_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class SSkipError(RuntimeError):
@@ -65,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L.sskip_attn_decode.argtypes = dec + [P]
         L.sskip_attn_decode_ex.restype = I
         L.sskip_attn_decode_ex.argtypes = dec + [P, P]
+        L.sskip_attn_decode_noalloc.restype = I
+        L.sskip_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, F, I, I, P, P]
         L.sskip_get_status.restype = I
         L.sskip_get_status.argtypes = [P]
         L.sskip_selftest_watchdog.restype = I
@@ -138,6 +143,24 @@ def sskip_attn_decode(q, kcache, vcache, seqlens, o, lse, *, sm_scale: float,
                                     _ptr(workspace), ws_bytes, _ptr(skip_count), _ptr(tile_state),
                                     _stream(stream))
     _check(rc, "sskip_attn_decode")
+
+
+def sskip_attn_decode_noalloc(q, kcache, vcache, seqlens, o, lse, *, sm_scale: float,
+                              threshold_scale_factor: float, Bc: int = 64, num_splits: int = 16,
+                              skip_count=None, stream=None) -> None:
+    """Marshal the same tensors as sskip_attn_decode, minus the workspace, into
+    sskip_attn_decode_noalloc: for callers that cannot allocate device memory,
+    the library's own fixed scratch array (DECODE_NOALLOC_SCRATCH_BYTES) holds
+    the split partials. Calls that overlap on the GPU race on that array."""
+    for t in (q, kcache, vcache, o):
+        _bf16_view(t)
+    B, Hq, d = q.shape
+    Hkv, Lmax = kcache.shape[1], kcache.shape[2]
+    rc = lib().sskip_attn_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens),
+                                         _ptr(o), _ptr(lse), B, Hq, Hkv, Lmax, d, float(sm_scale),
+                                         float(threshold_scale_factor), int(Bc), int(num_splits),
+                                         _ptr(skip_count), _stream(stream))
+    _check(rc, "sskip_attn_decode_noalloc")
 
 
 def sskip_get_status(stream=None) -> int:

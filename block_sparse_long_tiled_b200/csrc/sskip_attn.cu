@@ -304,3 +304,52 @@ SSKIP_API int sskip_selftest_watchdog(unsigned int limit_us, void* stream) {
   watchdog_selftest_kernel<<<1, 32, 0, st>>>((uint64_t)limit_us * 1000ull);
   return cudaGetLastError() == cudaSuccess ? SSKIP_OK : SSKIP_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------------------
+// Decode without any allocation by the caller.
+//
+// Some callers cannot call cudaMalloc at all -- embedded runtimes without a
+// device allocator, plugins whose host framework owns every device
+// allocation, serving loops that forbid allocation after start-up -- yet the
+// split-KV decode needs scratch for its per-split partial results.  For them the scratch lives in one fixed
+// device array of this library.  Every GPU that loads the library reserves it
+// for the life of the process.
+namespace sskip {
+namespace {
+
+static __device__ __align__(256) unsigned char g_decode_scratch[SSKIP_DECODE_NOALLOC_SCRATCH_BYTES];
+
+// The host-side name g_decode_scratch is only a stand-in for the device array;
+// its device address is looked up once per device, with that device current.
+void* decode_scratch_on_current_device() {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  const int dev = current_device();
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+}  // namespace sskip
+
+SSKIP_API int sskip_attn_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                                        const int* seqlens, void* o, float* lse, int B, int Hq,
+                                        int Hkv, int Lmax, int d, float sm_scale,
+                                        float threshold_scale_factor, int Bc, int num_splits,
+                                        unsigned long long* skip_count, void* stream) {
+  const size_t need = sskip_attn_decode_workspace_size(B, Hq, d, num_splits);
+  if (need == 0) return SSKIP_ERR_INVALID_ARG;
+  if (need > (size_t)SSKIP_DECODE_NOALLOC_SCRATCH_BYTES) return SSKIP_ERR_UNSUPPORTED;
+  void* scratch = decode_scratch_on_current_device();
+  if (!scratch) return SSKIP_ERR_CUDA;
+  return sskip_attn_decode_ex(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Lmax, d, sm_scale,
+                              threshold_scale_factor, Bc, num_splits, scratch,
+                              (size_t)SSKIP_DECODE_NOALLOC_SCRATCH_BYTES, skip_count, nullptr,
+                              stream);
+}

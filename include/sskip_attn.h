@@ -144,6 +144,42 @@ int sskip_attn_decode_ex(const void* q, const void* kcache, const void* vcache,
                          unsigned long long* skip_count, uint8_t* tile_state, void* stream);
 
 /*
+ * Decode for callers that cannot allocate device memory.  The paper has no
+ * counterpart: this is a deployment variant of sskip_attn_decode.
+ *
+ * Who needs it: code that must not call cudaMalloc -- embedded runtimes
+ * without a device allocator, plugins whose host framework owns every device
+ * allocation, latency-critical serving loops that forbid allocation after
+ * start-up.  The split-KV
+ * decode needs scratch for its per-split partial results; here that scratch is
+ * one fixed device array inside this library of
+ * SSKIP_DECODE_NOALLOC_SCRATCH_BYTES (32 MiB), reserved on every GPU that loads
+ * the library until the process exits.  The caller still passes inputs and
+ * outputs exactly as for sskip_attn_decode; everything else is the same.
+ *
+ *  - Returns SSKIP_ERR_UNSUPPORTED when the call would need more scratch than
+ *    the array holds, i.e. when
+ *    sskip_attn_decode_workspace_size(B, Hq, d, num_splits) exceeds
+ *    SSKIP_DECODE_NOALLOC_SCRATCH_BYTES (for example B = 64, Hq = 32, d = 128,
+ *    16 splits needs 16.9 MB and fits).
+ *  - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any
+ *    stream capture begins.
+ *  - Every call shares the one array, which keeps the last call's contents
+ *    (the kernels overwrite all of it they read).  Calls that overlap on the
+ *    GPU -- on different streams, or from different threads -- race on it and
+ *    give undefined results: serialise them.
+ */
+#define SSKIP_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+int sskip_attn_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                              const int* seqlens, void* o, float* lse,
+                              int B, int Hq, int Hkv, int Lmax, int d, float sm_scale,
+                              float threshold_scale_factor, int Bc, int num_splits,
+                              unsigned long long* skip_count, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's status
  * word: SSKIP_OK, or the first device-side error latched since the last call
  * (SSKIP_ERR_TIMEOUT when a bounded wait inside a kernel ran out; the kernel
