@@ -8,14 +8,19 @@
 // avoids loading the V blocks).
 //
 // Decode is HBM-bound (about 4 FLOP per cache byte), so the two contractions
-// run on CUDA cores and the design effort goes into keeping HBM busy:
-//   * K tiles stream through a 3-stage ring of 1-D bulk-async copies issued
-//     NK tiles ahead;
-//   * a skip decision needs only the K side (the running maximum after tile j
-//     depends on the local maxima of tiles <= j alone), so the vote for tile
-//     t is taken as soon as S_t exists and the V copy of a kept tile is issued
-//     immediately, LAG tiles before its P.V is consumed;
-//   * P.V for tile t - LAG overlaps the K copies and the votes of later tiles.
+// run on CUDA cores and the design keeps HBM busy and the per-tile critical
+// path short:
+//   * K tiles stream through a ring of 1-D bulk-async copies issued NK tiles
+//     ahead;
+//   * each of the 8 warps scores 8 of the tile's 64 keys (8 lanes per key, a
+//     transpose-reduce leaves one head's dot product per lane) and publishes
+//     its per-head maxima; after ONE block barrier every warp reads the eight
+//     maxima and takes the same joint decision itself -- no warp waits on a
+//     voting warp;
+//   * the V copy of a kept tile is issued right after that barrier, LAG tiles
+//     before its P.V runs (a decision needs only the K side);
+//   * each warp keeps P, its partial row sums and its partial O for its own
+//     keys, so P never crosses warps; the partials merge once per split.
 // The split's normalised partial O_s and lse_s (fp32) go to the workspace; a
 // second kernel merges the splits by log-sum-exp.
 #pragma once
@@ -43,26 +48,26 @@ struct DecodeParams {
 
 constexpr int kDecBc = 64;
 constexpr int kDecThreads = 256;
+constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kDecNK = 3;    // K ring stages
-constexpr int kDecLag = 2;   // P.V runs this many tiles behind the vote
+constexpr int kDecLag = 2;   // P.V runs this many tiles behind the decision
 constexpr int kDecNV = 3;    // V ring stages (> kDecLag)
-// S/P ring: phase A of tile t+1 may run in one warp while another warp still
-// reads P of tile t-LAG in phase D, so the ring needs LAG + 2 slots.
-constexpr int kDecNSB = kDecLag + 2;
+constexpr int kDecNPB = kDecLag + 1;  // per-warp P ring
+constexpr int kDecKeysPerWarp = kDecBc / kDecWarps;  // 8
 
 template <int D, int G>
 struct DecodeSmem {
   static constexpr int kTileBytes = kDecBc * D * 2;
   static constexpr int kK = 0;
   static constexpr int kV = kK + kDecNK * kTileBytes;
-  static constexpr int kS = kV + kDecNV * kTileBytes;                // [NSB][Bc][G] f32
-  static constexpr int kMeta = kS + kDecNSB * kDecBc * G * 4;         // alpha [NSB][G], kept [NSB]
-  static constexpr int kBar = (kMeta + kDecNSB * G * 4 + kDecNSB * 4 + 15) / 16 * 16;
-  static constexpr int kL = kBar + (kDecNK + kDecNV) * 8;             // l[G], m[G]
-  static constexpr int kAbort = kL + 2 * G * 4;
-  static constexpr int kTotal = kAbort + 16;
+  static constexpr int kP = kV + kDecNV * kTileBytes;                        // [W][NPB][8][G]
+  static constexpr int kAlpha = kP + kDecWarps * kDecNPB * kDecKeysPerWarp * G * 4;  // [W][NPB][G]
+  static constexpr int kWmax = kAlpha + kDecWarps * kDecNPB * G * 4;        // [2][G][W]
+  static constexpr int kLsum = kWmax + 2 * G * kDecWarps * 4;               // [W][G]
+  static constexpr int kBar = (kLsum + kDecWarps * G * 4 + 15) / 16 * 16;
+  static constexpr int kTotal = kBar + (kDecNK + kDecNV) * 8 + 16;
   // The cross-warp reduction of O at the end reuses the K ring.
-  static_assert(8 * G * D * 4 <= kDecNK * kTileBytes, "reduction scratch must fit in the K ring");
+  static_assert(kDecWarps * G * D * 4 <= kDecNK * kTileBytes, "reduction scratch fits the K ring");
 };
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float (&f)[8]) {
@@ -74,12 +79,44 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float (&f)[8]) {
   }
 }
 
+// Reduce G partial dot products over the 8 lanes of a key group so that lane
+// `sub` ends with the full sum for head sub / (8 / G): at each halving step a
+// lane keeps the half of the heads selected by its lane bit and receives the
+// partner's partials of that half; once one head is left the remaining lane
+// bits all-reduce it.
+template <int G>
+__device__ __forceinline__ float transpose_reduce8(const float (&acc)[G], int sub) {
+  float v[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) v[g] = acc[g];
+  int width = G;
+#pragma unroll
+  for (int m = 4; m >= 1; m >>= 1) {
+    if (width > 1) {
+      const int half = width / 2;
+      const bool upper = (sub & m) != 0;
+#pragma unroll
+      for (int i = 0; i < (G > 1 ? G / 2 : 1); ++i) {
+        if (i < half) {
+          const float send = upper ? v[i] : v[i + half];
+          const float keep = upper ? v[i + half] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+      }
+      width = half;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+    }
+  }
+  return v[0];
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const DecodeParams p) {
   using L = DecodeSmem<D, G>;
-  constexpr int PIECES = D / 8;          // 16-byte pieces per cache row
-  constexpr int PPL = PIECES / 8;        // pieces per lane (8 lanes per key)
-  constexpr int EPL = D / 32;            // P.V output elements per lane
+  constexpr int PPL = D / 64;        // 16-byte pieces per lane per key (8 lanes per key)
+  constexpr int EPL = D / 32;        // P.V output elements per lane
+  constexpr int LPH = 8 / G;         // lanes per head after the transpose-reduce
   extern __shared__ __align__(1024) uint8_t smem[];
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -98,13 +135,13 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
     return;
   }
 
-  float* Sbuf = reinterpret_cast<float*>(smem + L::kS);
-  float* alpha_s = reinterpret_cast<float*>(smem + L::kMeta);
-  int* kept_s = reinterpret_cast<int*>(smem + L::kMeta + kDecNSB * G * 4);
+  float* Pbuf = reinterpret_cast<float*>(smem + L::kP) + warp * kDecNPB * kDecKeysPerWarp * G;
+  float* Abuf = reinterpret_cast<float*>(smem + L::kAlpha) + warp * kDecNPB * G;
+  float* wmax = reinterpret_cast<float*>(smem + L::kWmax);
+  float* lsum = reinterpret_cast<float*>(smem + L::kLsum);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  float* l_s = reinterpret_cast<float*>(smem + L::kL);
-  float* m_s = l_s + G;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  volatile int* abort_flag =
+      reinterpret_cast<volatile int*>(smem + L::kBar + (kDecNK + kDecNV) * 8);
   const uint32_t k_smem = smem_u32(smem + L::kK);
   const uint32_t v_smem = smem_u32(smem + L::kV);
   auto kfull = [&](int s) { return smem_u32(&bars[s]); };
@@ -122,32 +159,26 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
   }
   __syncthreads();
 
-  auto issue_k = [&](int t) {
-    const int keys = tile_keys(t);
-    const uint32_t bytes = (uint32_t)keys * D * 2;
-    const int s = t % kDecNK;
-    mbar_arrive_expect_tx(kfull(s), bytes);
-    bulk_load(k_smem + s * L::kTileBytes, kbase + (size_t)(j0 + t) * kDecBc * D, bytes, kfull(s));
+  auto issue = [&](uint32_t ring, int stage, uint32_t bar, const __nv_bfloat16* base, int t) {
+    const uint32_t bytes = (uint32_t)tile_keys(t) * D * 2;
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(ring + stage * L::kTileBytes, base + (size_t)(j0 + t) * kDecBc * D, bytes, bar);
   };
-  auto issue_v = [&](int t) {
-    const int keys = tile_keys(t);
-    const uint32_t bytes = (uint32_t)keys * D * 2;
-    const int s = t % kDecNV;
-    mbar_arrive_expect_tx(vfull(s), bytes);
-    bulk_load(v_smem + s * L::kTileBytes, vbase + (size_t)(j0 + t) * kDecBc * D, bytes, vfull(s));
-  };
-
   if (tid == 0)
-    for (int t = 0; t < min(kDecNK, ntiles); ++t) issue_k(t);
+    for (int t = 0; t < min(kDecNK, ntiles); ++t) issue(k_smem, t, kfull(t), kbase, t);
 
-  // This thread's slice of the G query rows: pieces (lane % 8) + 8 * i.
-  const int cc = lane & 7;
+  // Lane layout of the scores: 8 lanes per key (sub = lane % 8), 4 keys per
+  // warp per pass; pass ps covers keys ps*32 + warp*4 + lane/8.
+  const int sub = lane & 7, kq = lane >> 3;
+  const int hs = sub / LPH;             // head whose score this lane holds
+  const bool owner = (sub % LPH) == 0;  // one writer per (key, head)
+  const int hv = lane % G;              // head this lane votes / keeps state for
   float qreg[G][PPL * 8];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int i = 0; i < PPL; ++i) {
-      const uint4 w = *reinterpret_cast<const uint4*>(p.q + (head0 + g) * D + (cc + 8 * i) * 8);
+      const uint4 w = *reinterpret_cast<const uint4*>(p.q + (head0 + g) * D + (sub + 8 * i) * 8);
       float f[8];
       bf16x8_to_f32(w, f);
 #pragma unroll
@@ -156,35 +187,37 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
 
   const bool t_positive = p.tsf > 0.f;
   const float log2_t = t_positive ? (float)log2((double)p.tsf / (double)Lb) : -INFINITY;
-  // Warp 0 owns the online-softmax state of the G rows (replicated per lane).
-  float m_run[G], l_run[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) { m_run[g] = -INFINITY; l_run[g] = 0.f; }
+  float m_run = -INFINITY;  // running max of head hv (identical in every warp)
+  float l_lane = 0.f;       // this lane's share of the row sum of head hs
   float oacc[G][EPL];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int e = 0; e < EPL; ++e) oacc[g][e] = 0.f;
-  uint32_t v_phase = 0;  // one parity bit per V slot
+  uint32_t v_phase = 0;      // one parity bit per V slot
+  uint64_t kept_mask = 0;    // bit (t % 64): tile t was kept
   int n_skipped = 0;
 
   for (int t = 0; t < ntiles + kDecLag; ++t) {
-    if (t < ntiles) {
-      // ---- S_t = q K_t^T (scaled to log2 units); keys past L_b are -inf.
-      const int s = t % kDecNK;
-      mbar_wait(kfull(s), (t / kDecNK) & 1, abort_flag);
+    float s[2] = {-INFINITY, -INFINITY};
+    const bool live = t < ntiles;
+    if (live) {
+      // ---- scores of this warp's 8 keys, in log2 units; keys past L_b -> -inf.
+      const int ks = t % kDecNK;
+      mbar_wait(kfull(ks), (t / kDecNK) & 1, abort_flag);
       const int keys = tile_keys(t);
-      const uint8_t* ktile = smem + L::kK + s * L::kTileBytes;
-      float* St = Sbuf + (t % kDecNSB) * kDecBc * G;
+      const uint8_t* ktile = smem + L::kK + ks * L::kTileBytes;
+      float mx = -INFINITY;
 #pragma unroll
-      for (int ps = 0; ps < kDecBc / 32; ++ps) {
-        const int key = ps * 32 + warp * 4 + (lane >> 3);
+      for (int ps = 0; ps < 2; ++ps) {
+        const int key = ps * 32 + warp * 4 + kq;
         float acc[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) acc[g] = 0.f;
 #pragma unroll
         for (int i = 0; i < PPL; ++i) {
-          const uint4 w = *reinterpret_cast<const uint4*>(ktile + key * D * 2 + (cc + 8 * i) * 16);
+          const uint4 w =
+              *reinterpret_cast<const uint4*>(ktile + key * D * 2 + (sub + 8 * i) * 16);
           float f[8];
           bf16x8_to_f32(w, f);
 #pragma unroll
@@ -192,88 +225,70 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc[g] = fmaf(qreg[g][i * 8 + e], f[e], acc[g]);
         }
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 1);
-          acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 2);
-          acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 4);
-        }
-        if (cc < G) {
-          float v = acc[0];
-#pragma unroll
-          for (int g = 1; g < G; ++g) v = (cc == g) ? acc[g] : v;
-          St[key * G + cc] = (key < keys) ? v * p.scale_log2 : -INFINITY;
-        }
+        const float dot = transpose_reduce8<G>(acc, sub);
+        s[ps] = (key < keys) ? dot * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, s[ps]);
       }
+      // per-head max over the warp's 4 key groups (lane bits 3, 4)
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      if (kq == 0 && owner) wmax[((t & 1) * G + hs) * kDecWarps + warp] = mx;
     }
-    __syncthreads();  // S_t complete; K slot t % NK free; P.V of t-1-LAG done
+    __syncthreads();  // maxima of tile t published; K slot t % NK free; P.V of t-1-LAG done
 
-    if (t < ntiles) {
-      if (tid == 0 && t + kDecNK < ntiles && !*abort_flag) issue_k(t + kDecNK);
-      if (warp == 0) {
-        // ---- joint vote of the G rows, then the online-softmax update.
-        float* St = Sbuf + (t % kDecNSB) * kDecBc * G;
-        float s0[G], s1[G], mloc[G];
+    if (live) {
+      if (tid == 0 && t + kDecNK < ntiles && !*abort_flag)
+        issue(k_smem, (t + kDecNK) % kDecNK, kfull((t + kDecNK) % kDecNK), kbase, t + kDecNK);
+      // ---- the joint decision, taken identically by every warp.
+      const float* wm = wmax + ((t & 1) * G + hv) * kDecWarps;
+      float m_loc = wm[0];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          s0[g] = St[lane * G + g];
-          s1[g] = St[(lane + 32) * G + g];
-          float mx = fmaxf(s0[g], s1[g]);
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-          mloc[g] = mx;
+      for (int w = 1; w < kDecWarps; ++w) m_loc = fmaxf(m_loc, wm[w]);
+      const bool skip =
+          __all_sync(0xffffffffu, row_passes_log2(m_loc, m_run, log2_t, t_positive));
+      if (!skip) {
+        const float m_new = fmaxf(m_run, m_loc);
+        const float a = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
+        m_run = m_new;
+        const float mh = __shfl_sync(0xffffffffu, m_new, hs);  // lane hs holds head hs
+        const float ah = __shfl_sync(0xffffffffu, a, hs);
+        const float p0 = ex2_approx(s[0] - mh), p1 = ex2_approx(s[1] - mh);
+        l_lane = ah * l_lane + p0 + p1;
+        float* Pt = Pbuf + (t % kDecNPB) * kDecKeysPerWarp * G;
+        if (owner) {
+          Pt[kq * G + hs] = p0;
+          Pt[(4 + kq) * G + hs] = p1;
         }
-        bool skip = true;
-#pragma unroll
-        for (int g = 0; g < G; ++g) skip = skip && row_passes_log2(mloc[g], m_run[g], log2_t, t_positive);
-        if (!skip) {
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float m_new = fmaxf(m_run[g], mloc[g]);
-            const float a = (m_run[g] == -INFINITY) ? 0.f : ex2_approx(m_run[g] - m_new);
-            const float p0 = ex2_approx(s0[g] - m_new);
-            const float p1 = ex2_approx(s1[g] - m_new);
-            St[lane * G + g] = p0;
-            St[(lane + 32) * G + g] = p1;
-            float sum = p0 + p1;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-            l_run[g] = a * l_run[g] + sum;
-            m_run[g] = m_new;
-            if (lane == 0) alpha_s[(t % kDecNSB) * G + g] = a;
-          }
-        }
-        if (lane == 0) {
-          kept_s[t % kDecNSB] = skip ? 0 : 1;
-          n_skipped += skip ? 1 : 0;
-          if (p.tile_state)
-            p.tile_state[((size_t)b * p.Hkv + kvh) * p.n_k_max + j0 + t] = skip ? 2 : 1;
-          // The V copy of a kept tile goes out now; its slot was last read by
-          // the P.V of tile t - NV, which finished before the barrier above.
-          if (!skip && !*abort_flag) issue_v(t);
-        }
+        if (lane < G) Abuf[(t % kDecNPB) * G + lane] = a;
+        kept_mask |= 1ull << (t & 63);
+        if (tid == 0 && !*abort_flag) issue(v_smem, t % kDecNV, vfull(t % kDecNV), vbase, t);
+      } else {
+        kept_mask &= ~(1ull << (t & 63));
+        n_skipped += 1;
       }
+      if (tid == 0 && p.tile_state)
+        p.tile_state[((size_t)b * p.Hkv + kvh) * p.n_k_max + j0 + t] = skip ? 2 : 1;
     }
-    __syncthreads();  // decision, P and alpha of tile t visible
 
     const int u = t - kDecLag;
-    if (u >= 0 && kept_s[u % kDecNSB]) {
-      // ---- O = alpha O + P_u V_u over this warp's keys {warp + 8 i}.
+    if (u >= 0 && ((kept_mask >> (u & 63)) & 1)) {
+      // ---- O = alpha O + P_u V_u over this warp's 8 keys.
       const int vs = u % kDecNV;
       mbar_wait(vfull(vs), (v_phase >> vs) & 1, abort_flag);
       v_phase ^= 1u << vs;
+      __syncwarp();
       const int keys = tile_keys(u);
-      const float* Pu = Sbuf + (u % kDecNSB) * kDecBc * G;
+      const float* Pu = Pbuf + (u % kDecNPB) * kDecKeysPerWarp * G;
       const uint8_t* vtile = smem + L::kV + vs * L::kTileBytes;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float a = alpha_s[(u % kDecNSB) * G + g];
+        const float a = Abuf[(u % kDecNPB) * G + g];
 #pragma unroll
         for (int e = 0; e < EPL; ++e) oacc[g][e] *= a;
       }
 #pragma unroll
-      for (int i = 0; i < kDecBc / 8; ++i) {
-        const int key = warp + 8 * i;
+      for (int k = 0; k < kDecKeysPerWarp; ++k) {
+        const int key = (k >> 2) * 32 + warp * 4 + (k & 3);
         if (key < keys) {
           float vf[EPL];
           if constexpr (EPL == 4) {
@@ -289,7 +304,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
           }
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            const float pk = Pu[key * G + g];
+            const float pk = Pu[k * G + g];
 #pragma unroll
             for (int e = 0; e < EPL; ++e) oacc[g][e] = fmaf(pk, vf[e], oacc[g][e]);
           }
@@ -298,31 +313,40 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
     }
   }
 
-  // ---- epilogue: reduce the 8 warps' partial O, normalise, write the split.
-  __syncthreads();
+  // ---- epilogue: merge the warps' partial O and row sums, write the split.
+  // A lane's row-sum share counts once per (key group, head).
+  float lw = owner ? l_lane : 0.f;
+  lw += __shfl_xor_sync(0xffffffffu, lw, 8);
+  lw += __shfl_xor_sync(0xffffffffu, lw, 16);
+  __syncthreads();  // every warp is past its last use of the K ring
   float* red = reinterpret_cast<float*>(smem + L::kK);
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int e = 0; e < EPL; ++e) red[(warp * G + g) * D + lane * EPL + e] = oacc[g][e];
-  if (warp == 0 && lane == 0) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) { l_s[g] = l_run[g]; m_s[g] = m_run[g]; }
-    if (p.counts) {
-      atomicAdd(&p.counts[0], (unsigned long long)n_skipped);
-      atomicAdd(&p.counts[1], (unsigned long long)ntiles);
-    }
+  if (kq == 0 && owner) lsum[warp * G + hs] = lw;
+  if (tid == 0 && p.counts) {
+    atomicAdd(&p.counts[0], (unsigned long long)n_skipped);
+    atomicAdd(&p.counts[1], (unsigned long long)ntiles);
   }
   __syncthreads();
   for (int i = tid; i < G * D; i += kDecThreads) {
     const int g = i / D, e = i % D;
-    float acc = 0.f;
+    float acc = 0.f, l = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) acc += red[(w * G + g) * D + e];
-    p.o_part[((head0 + g) * p.S + split) * D + e] = acc / l_s[g];
+    for (int w = 0; w < kDecWarps; ++w) {
+      acc += red[(w * G + g) * D + e];
+      l += lsum[w * G + g];
+    }
+    p.o_part[((head0 + g) * p.S + split) * D + e] = acc / l;
   }
-  if (tid < G)
-    p.lse_part[(head0 + tid) * p.S + split] = (m_s[tid] + __log2f(l_s[tid])) * 0.69314718055994531f;
+  if (tid < G) {
+    float l = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) l += lsum[w * G + tid];
+    // lanes tid < G of warp 0 hold the running max of head tid
+    p.lse_part[(head0 + tid) * p.S + split] = (m_run + __log2f(l)) * 0.69314718055994531f;
+  }
 }
 
 // Merge the splits of one (batch, query head): lse = log sum_s exp(lse_s),
