@@ -82,7 +82,7 @@ def load_peaks() -> tuple[dict, str]:
 
 
 KERNEL_SOURCES = {
-    "prefill_kernel": ("prefill_sm100.cuh", "sm100_ptx.cuh", "skip_rule.cuh"),
+    "prefill_kernel": ("prefill_sm100.cuh", "sm100_ptx.cuh", "sm100_tmem.cuh", "skip_rule.cuh"),
     "decode_split_kernel": ("decode_sm100.cuh", "sm100_ptx.cuh", "skip_rule.cuh"),
 }
 

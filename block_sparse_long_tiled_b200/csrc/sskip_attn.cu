@@ -154,7 +154,7 @@ SSKIP_API int sskip_attn_prefill_ex(const void* q, const void* k, const void* v,
     return SSKIP_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return SSKIP_ERR_UNSUPPORTED;
   if (!((Br == 64 && Bc == 64) || (Br == 128 && Bc == 128))) return SSKIP_ERR_UNSUPPORTED;
-  const long long n_units = (L + 127) / 128;
+  const long long n_units = (L + kPfUnitRows - 1) / kPfUnitRows;
   if ((long long)B * Hq * n_units >= (1ll << 31) || (long long)B * Hq >= (1ll << 31))
     return SSKIP_ERR_UNSUPPORTED;
 
