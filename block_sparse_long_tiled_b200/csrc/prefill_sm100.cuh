@@ -17,9 +17,9 @@
 //               NK-stage ring (K is needed for every visited tile).
 //   warp 1      TMEM allocator; one thread issues every tcgen05.mma:
 //               per key tile j: P_A.V_j, S_A(j+1), P_B.V_j, S_B(j+1).
-//   warp 2      V producer: collects both warpgroups' votes on tile j and
-//               issues the V_j TMA as soon as either keeps the tile; a tile
-//               both skip never loads V.
+//   warp 2      V producer: watches both warpgroups' votes on tile j and
+//               issues the V_j TMA on the first "keep"; a tile both skip
+//               never loads V.
 //   warps 4..7  softmax of tile A, thread r = TMEM lane r = query row r.
 //   warps 8..11 softmax of tile B.
 // A softmax warpgroup, per key tile: loads its S row from TMEM, masks it,
@@ -62,6 +62,29 @@ constexpr int kPfUnitRows = 256;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kPfVoteSlots = 4;
 
+// Tuning switches of the softmax inner loop (compile-time).
+#ifndef SSKIP_PF_FMA_EXP
+#define SSKIP_PF_FMA_EXP 0   // element pairs per 8 whose exp2 runs on the FMA pipe
+#endif
+#ifndef SSKIP_PF_PACK_PRMT
+#define SSKIP_PF_PACK_PRMT 0  // bf16 packing by byte permute instead of cvt
+#endif
+#ifndef SSKIP_PF_SCALAR
+#define SSKIP_PF_SCALAR 0     // scalar instead of packed f32x2 scale / sum
+#endif
+constexpr int kExp2FmaPairsPer8 = SSKIP_PF_FMA_EXP;
+__device__ __forceinline__ constexpr bool exp2_on_fma(int pair) {
+  return kExp2FmaPairsPer8 > 0 && ((pair & 7) * kExp2FmaPairsPer8) % 8 < kExp2FmaPairsPer8;
+}
+// Byte-permute packing rounds each (non-negative) P to bf16 half-up: add half
+// a bf16 unit in the last place to the fp32 bits, keep the top 16 bits.  It
+// differs from round-to-nearest-even only at exact ties and runs on the
+// integer ALU instead of the conversion unit.
+__device__ __forceinline__ uint32_t pack_bf16x2_halfup(float lo, float hi) {
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
+}
+constexpr float kPackBias = 0.0f;
+
 template <int D, int BC>
 struct PrefillCfg {
   static constexpr bool kBig = (D * BC >= 128 * 128);
@@ -74,8 +97,8 @@ struct PrefillCfg {
   static constexpr int kV = kK + kNK * kKVBytes;
   static constexpr int kBar = kV + kNV * kKVBytes;
   // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2],
-  // dec[2], votes_full[VS], votes_empty[VS], mma_done
-  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 2 * kPfVoteSlots + 1;
+  // dec[2], vote_full[2][VS], vote_empty[2][VS], mma_done
+  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 4 * kPfVoteSlots + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   // dec_kept[2], vote_kept[VS][2], warp vote flags [2 wg][2 parity][4], tmem, abort
   static constexpr int kMiscInts = 2 + 2 * kPfVoteSlots + 16 + 2;
@@ -117,9 +140,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   auto b_vempty = [&](int s) { return smem_u32(&bars[1 + 2 * NK + NV + s]); };
   auto b_sfull = [&](int w) { return smem_u32(&bars[1 + 2 * NK + 2 * NV + w]); };
   auto b_dec = [&](int w) { return smem_u32(&bars[1 + 2 * NK + 2 * NV + 2 + w]); };
-  auto b_vfull_vote = [&](int s) { return smem_u32(&bars[1 + 2 * NK + 2 * NV + 4 + s]); };
-  auto b_vempty_vote = [&](int s) { return smem_u32(&bars[1 + 2 * NK + 2 * NV + 4 + VS + s]); };
-  const uint32_t b_mmadone = smem_u32(&bars[1 + 2 * NK + 2 * NV + 4 + 2 * VS]);
+  auto b_vote_full = [&](int w, int s) { return smem_u32(&bars[1 + 2 * NK + 2 * NV + 4 + w * VS + s]); };
+  auto b_vote_empty = [&](int w, int s) {
+    return smem_u32(&bars[1 + 2 * NK + 2 * NV + 4 + 2 * VS + w * VS + s]);
+  };
+  const uint32_t b_mmadone = smem_u32(&bars[1 + 2 * NK + 2 * NV + 4 + 4 * VS]);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -152,7 +177,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int s = 0; s < NK; ++s) { mbar_init(b_kfull(s), 1); mbar_init(b_kempty(s), 1); }
     for (int s = 0; s < NV; ++s) { mbar_init(b_vfull(s), 1); mbar_init(b_vempty(s), 1); }
     for (int w = 0; w < 2; ++w) { mbar_init(b_sfull(w), 1); mbar_init(b_dec(w), 1); }
-    for (int s = 0; s < VS; ++s) { mbar_init(b_vfull_vote(s), 2); mbar_init(b_vempty_vote(s), 1); }
+    for (int w = 0; w < 2; ++w)
+      for (int s = 0; s < VS; ++s) { mbar_init(b_vote_full(w, s), 1); mbar_init(b_vote_empty(w, s), 1); }
     mbar_init(b_mmadone, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -167,7 +193,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 4) {
-    regs_dealloc<56>();
+    regs_dealloc<80>();
     if (warp == 0 && lane == 0) {
       // ================= TMA producer: Q_A, Q_B, then the K ring ==========
       tma_prefetch_desc(&tmQ);
@@ -198,15 +224,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
     } else if (warp == 1 && lane == 0) {
       // ================= MMA issuer =================
+      // Descriptors are built once per operand; a K step only moves the start
+      // address field (bits 0-13, in 16-byte units), which never carries out
+      // of it since shared addresses stay below 256 KB.
+      const uint64_t dq0 = smem_desc_sw128(sbase + C::kQ, 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(sbase + C::kK, 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(sbase + C::kV, BC * 128, 1024);
       auto issue_s = [&](int w, int j) {
-        const int s = j % NK;
+        const uint64_t da = dq0 + (uint64_t)((w * C::kQBytes) >> 4);
+        const uint64_t db = dk0 + (uint64_t)(((j % NK) * C::kKVBytes) >> 4);
         const uint32_t d_tmem = tmem + w * BC;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a = sbase + C::kQ + w * C::kQBytes + (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          const uint32_t bk = sbase + C::kK + s * C::kKVBytes + (kk >> 2) * (BC * 128) + (kk & 3) * 32;
-          umma_ss(d_tmem, smem_desc_sw128(a, 16, 1024), smem_desc_sw128(bk, 16, 1024), IDESC_S,
-                  kk > 0 ? 1u : 0u);
+          const uint32_t oa = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+          const uint32_t ob = ((kk >> 2) * (BC * 128) + (kk & 3) * 32) >> 4;
+          umma_ss(d_tmem, da + oa, db + ob, IDESC_S, kk > 0 ? 1u : 0u);
         }
         umma_commit(b_sfull(w));
       };
@@ -214,12 +246,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       auto issue_pv = [&](int w, int vs) {
         const uint32_t p_tmem = tmem + w * BC;
         const uint32_t o_tmem = tmem + 2 * BC + w * D;
+        const uint64_t dv = dv0 + (uint64_t)((vs * C::kKVBytes) >> 4);
+        const uint32_t acc0 = pv_count[w] > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < BC / 16; ++kk) {
-          const uint32_t bv = sbase + C::kV + vs * C::kKVBytes + kk * 16 * 128;
-          umma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(bv, BC * 128, 1024), IDESC_PV,
-                  (pv_count[w] > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BC / 16; ++kk)
+          umma_ts(o_tmem, p_tmem + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), IDESC_PV,
+                  kk > 0 ? 1u : acc0);
         ++pv_count[w];
       };
       bool ok = mbar_wait(b_qfull, 0, abort_flag);
@@ -277,23 +309,48 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // Every MMA issued by this thread completes before the epilogue reads O.
       umma_commit(b_mmadone);
     } else if (warp == 2 && lane == 0) {
-      // ================= V producer: issues V_j once a warpgroup keeps j ====
+      // ================= V producer: issues V_j on the FIRST keep vote =====
+      // Each warpgroup posts its vote on tile j as soon as it has its row
+      // maxima; the first "keep" starts the V_j load, so its latency hides
+      // behind that warpgroup's exponentials.  Both votes are consumed in
+      // order to keep the slots' phases exact.
       tma_prefetch_desc(&tmV);
       int kc = 0, last = -1;
-      for (int j = 0; j < n_j; ++j) {
+      for (int j = 0; j < n_j && !*abort_flag; ++j) {
         const int vslot = j % VS;
-        if (!mbar_wait(b_vfull_vote(vslot), (j / VS) & 1, abort_flag)) break;
-        const bool keep = vote_kept[vslot * 2 + 0] != 0 || vote_kept[vslot * 2 + 1] != 0;
-        mbar_arrive(b_vempty_vote(vslot));
-        if (!keep || *abort_flag) continue;
-        const int vs = kc % NV;
-        if (kc >= NV && !mbar_wait(b_vempty(vs), ((kc / NV) - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(b_vfull(vs), C::kKVBytes);
+        const uint32_t par = (j / VS) & 1;
+        bool seen[2] = {false, false}, kept_any = false, issued = false;
+        const uint64_t t0 = globaltimer_ns();
+        while (!(seen[0] && seen[1])) {
+          bool progress = false;
 #pragma unroll
-        for (int blk = 0; blk < D / 64; ++blk)
-          tma_load_3d(sbase + C::kV + vs * C::kKVBytes + blk * BC * 128, &tmV, b_vfull(vs),
-                      blk * 64, j * BC, b * p.Hkv + kvh);
-        last = kc++;
+          for (int w = 0; w < 2; ++w) {
+            if (!seen[w] && mbar_test_wait(b_vote_full(w, vslot), par)) {
+              seen[w] = true;
+              progress = true;
+              kept_any = kept_any || vote_kept[vslot * 2 + w] != 0;
+              mbar_arrive(b_vote_empty(w, vslot));
+            }
+          }
+          if (!progress) __nanosleep(40);  // leave issue slots to the softmax warps
+          if (kept_any && !issued) {
+            const int vs = kc % NV;
+            if (kc >= NV && !mbar_wait(b_vempty(vs), ((kc / NV) - 1) & 1, abort_flag)) break;
+            mbar_arrive_expect_tx(b_vfull(vs), C::kKVBytes);
+#pragma unroll
+            for (int blk = 0; blk < D / 64; ++blk)
+              tma_load_3d(sbase + C::kV + vs * C::kKVBytes + blk * BC * 128, &tmV, b_vfull(vs),
+                          blk * 64, j * BC, b * p.Hkv + kvh);
+            issued = true;
+            last = kc++;
+          }
+          if (*abort_flag) break;
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            latch_status(kStatusTimeout);
+            break;
+          }
+        }
       }
       if (*abort_flag) {
         int dummy = 0;
@@ -302,7 +359,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
     }
   } else {
-    regs_alloc<224>();
+    regs_alloc<208>();
     // ================= softmax warpgroups =================
     const int wg = (warp - 4) >> 2;  // 0: tile A, 1: tile B
     const int wq = warp & 3;         // TMEM lane quadrant
@@ -333,9 +390,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 
     auto post_vote = [&](int j, bool kept) {  // elected thread only
       const int vslot = j % VS;
-      if (j >= VS) mbar_wait(b_vempty_vote(vslot), ((j / VS) - 1) & 1, abort_flag);
+      if (j >= VS) mbar_wait(b_vote_empty(wg, vslot), ((j / VS) - 1) & 1, abort_flag);
       vote_kept[vslot * 2 + wg] = kept ? 1 : 0;
-      mbar_arrive(b_vfull_vote(vslot));
+      mbar_arrive(b_vote_full(wg, vslot));
     };
 
     for (int j = 0; j < n_j; ++j) {
@@ -415,21 +472,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         // P = exp2(S * scale - m_ref) for kept rows, 0 otherwise; bf16 pairs.
         const uint64_t scale2 = f2pack(scale, scale);
-        const float nref = mine ? -m_ref : -INFINITY;
+        const float nref = mine ? kPackBias - m_ref : -INFINITY;
         const uint64_t nref2 = f2pack(nref, nref);
-        uint64_t sum2 = f2pack(0.f, 0.f);
-        uint32_t pk[BC / 2];
-#pragma unroll
-        for (int c = 0; c < BC / 2; ++c) {
-          float x0, x1;
-          f2unpack(ffma2(f2pack(s[2 * c], s[2 * c + 1]), scale2, nref2), x0, x1);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          sum2 = fadd2(sum2, f2pack(p0, p1));
-          pk[c] = pack_bf16x2(p0, p1);
-        }
-        float sa, sb;
-        f2unpack(sum2, sa, sb);
-        l_run += mine ? (sa + sb) : 0.f;
         __syncwarp();
         if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
@@ -442,13 +486,42 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             tmem_st32(tO + c * 32, w32);
           }
         }
+        uint64_t sum2 = f2pack(0.f, 0.f);
+        float suma = 0.f, sumb = 0.f;
 #pragma unroll
-        for (int c = 0; c < BC / 64; ++c) {
-          uint32_t w32[32];
+        for (int h = 0; h < BC / 64; ++h) {  // 64 keys -> 32 packed columns at a time
+          uint32_t pk[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) w32[i] = pk[c * 32 + i];
-          tmem_st32(tS + c * 32, w32);
+          for (int i = 0; i < 32; ++i) {
+            const int c = h * 32 + i;
+            float p0, p1;
+            if (SSKIP_PF_SCALAR && !exp2_on_fma(c)) {
+              p0 = ex2_approx(fmaf(s[2 * c], scale, nref));
+              p1 = ex2_approx(fmaf(s[2 * c + 1], scale, nref));
+              suma += p0;
+              sumb += p1;
+            } else {
+              const uint64_t x2 = ffma2(f2pack(s[2 * c], s[2 * c + 1]), scale2, nref2);
+              if (exp2_on_fma(c)) {
+                f2unpack(exp2_fma2(x2), p0, p1);
+              } else {
+                float x0, x1;
+                f2unpack(x2, x0, x1);
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              sum2 = fadd2(sum2, f2pack(p0, p1));
+            }
+            if (SSKIP_PF_PACK_PRMT)
+              pk[i] = pack_bf16x2_halfup(p0, p1);
+            else
+              pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32(tS + h * 32, pk);
         }
+        float sa, sb;
+        f2unpack(sum2, sa, sb);
+        l_run += mine ? ((sa + sb) + (suma + sumb)) : 0.f;
         tmem_st_wait();
         tc_fence_before();
         named_bar_sync(bar_id, 128);
@@ -484,7 +557,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
     }
     if (store)
-      p.lse[((size_t)b * p.Hq + hq) * p.L + row] = (m_ref + __log2f(l_run)) * 0.69314718055994531f;
+      p.lse[((size_t)b * p.Hq + hq) * p.L + row] =
+          (m_ref - kPackBias + __log2f(l_run)) * 0.69314718055994531f;
     if (elected && p.counts) {
       atomicAdd(&p.counts[0], (unsigned long long)n_skip);
       atomicAdd(&p.counts[1], (unsigned long long)n_vis);

@@ -62,6 +62,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity. Returns false when the CTA
 // is aborting (another role gave up) or when this wait itself ran out.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
@@ -250,6 +263,33 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// 2^x for a pair of fp32 on the FMA pipe (offloads the MUFU unit).  Method
+// (Cody-Waite range reduction + a polynomial fitted here by
+// fit_exp2_poly.py): clamp x >= -126; n = round(x) by adding 1.5 * 2^23;
+// f = x - n in [-1/2, 1/2]; p(f) ~ 2^f by a degree-3 polynomial with minimax
+// relative error 8.4e-5; the result is p(f) * 2^n, made by adding n to the
+// exponent bits of p(f).  Whole-method relative error <= 1.7e-4 over
+// [-126, 8]; -inf maps to 2^-126 * p, i.e. effectively zero.
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  constexpr float kC0 = 0.999919593334198f, kC1 = 0.6932621598243713f;
+  constexpr float kC2 = 0.24271413683891296f, kC3 = 0.055212993174791336f;
+  float a, b;
+  f2unpack(x2, a, b);
+  const uint64_t xc = f2pack(fmaxf(a, -126.0f), fmaxf(b, -126.0f));
+  const uint64_t t2 = fadd2(xc, f2pack(kMagic, kMagic));
+  const uint64_t n2 = fadd2(t2, f2pack(-kMagic, -kMagic));
+  const uint64_t f2 = ffma2(n2, f2pack(-1.0f, -1.0f), xc);
+  uint64_t p2 = ffma2(f2pack(kC3, kC3), f2, f2pack(kC2, kC2));
+  p2 = ffma2(p2, f2, f2pack(kC1, kC1));
+  p2 = ffma2(p2, f2, f2pack(kC0, kC0));
+  float plo, phi, tlo, thi;
+  f2unpack(p2, plo, phi);
+  f2unpack(t2, tlo, thi);
+  return f2pack(__uint_as_float(__float_as_uint(plo) + (__float_as_uint(tlo) << 23)),
+                __uint_as_float(__float_as_uint(phi) + (__float_as_uint(thi) << 23)));
 }
 
 // Per-warpgroup register reallocation (counts must be multiples of 8 and the
