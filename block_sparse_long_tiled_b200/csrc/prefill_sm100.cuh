@@ -72,6 +72,12 @@ constexpr int kPfVoteSlots = 4;
 #ifndef SSKIP_PF_SCALAR
 #define SSKIP_PF_SCALAR 0     // scalar instead of packed f32x2 scale / sum
 #endif
+#ifndef SSKIP_PF_RELOAD
+#define SSKIP_PF_RELOAD 1     // reload S from TMEM in 64-column halves for the exponentials
+#endif
+#ifndef SSKIP_PF_NACC
+#define SSKIP_PF_NACC 4       // independent packed accumulators of the row sum
+#endif
 constexpr int kExp2FmaPairsPer8 = SSKIP_PF_FMA_EXP;
 __device__ __forceinline__ constexpr bool exp2_on_fma(int pair) {
   return kExp2FmaPairsPer8 > 0 && ((pair & 7) * kExp2FmaPairsPer8) % 8 < kExp2FmaPairsPer8;
@@ -486,22 +492,41 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             tmem_st32(tO + c * 32, w32);
           }
         }
-        uint64_t sum2 = f2pack(0.f, 0.f);
+        uint64_t sum2v[SSKIP_PF_NACC];
+#pragma unroll
+        for (int a = 0; a < SSKIP_PF_NACC; ++a) sum2v[a] = f2pack(0.f, 0.f);
         float suma = 0.f, sumb = 0.f;
 #pragma unroll
         for (int h = 0; h < BC / 64; ++h) {  // 64 keys -> 32 packed columns at a time
           uint32_t pk[32];
+          float* sh = s;
+          uint32_t rr[64];
+          if constexpr (SSKIP_PF_RELOAD) {
+            // The row max is known; re-read this half of S (its columns are
+            // still intact: P of half h lands in columns [32h, 32h + 32)).
+            tmem_ld32_async(tS + h * 64, rr);
+            tmem_ld32_async(tS + h * 64 + 32, rr + 32);
+            tmem_wait_ld_tie64(rr);
+            sh = reinterpret_cast<float*>(rr) - h * 64;
+            if (need_mask) {
+#pragma unroll
+              for (int c = 0; c < 64; ++c) {
+                const int key = key0 + h * 64 + c;
+                if (key >= p.L || (CAUSAL && key > row)) rr[c] = __float_as_uint(-INFINITY);
+              }
+            }
+          }
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int c = h * 32 + i;
             float p0, p1;
             if (SSKIP_PF_SCALAR && !exp2_on_fma(c)) {
-              p0 = ex2_approx(fmaf(s[2 * c], scale, nref));
-              p1 = ex2_approx(fmaf(s[2 * c + 1], scale, nref));
+              p0 = ex2_approx(fmaf(sh[2 * c], scale, nref));
+              p1 = ex2_approx(fmaf(sh[2 * c + 1], scale, nref));
               suma += p0;
               sumb += p1;
             } else {
-              const uint64_t x2 = ffma2(f2pack(s[2 * c], s[2 * c + 1]), scale2, nref2);
+              const uint64_t x2 = ffma2(f2pack(sh[2 * c], sh[2 * c + 1]), scale2, nref2);
               if (exp2_on_fma(c)) {
                 f2unpack(exp2_fma2(x2), p0, p1);
               } else {
@@ -510,7 +535,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 p0 = ex2_approx(x0);
                 p1 = ex2_approx(x1);
               }
-              sum2 = fadd2(sum2, f2pack(p0, p1));
+              sum2v[c % SSKIP_PF_NACC] = fadd2(sum2v[c % SSKIP_PF_NACC], f2pack(p0, p1));
             }
             if (SSKIP_PF_PACK_PRMT)
               pk[i] = pack_bf16x2_halfup(p0, p1);
@@ -519,6 +544,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
           tmem_st32(tS + h * 32, pk);
         }
+        uint64_t sum2 = sum2v[0];
+#pragma unroll
+        for (int a = 1; a < SSKIP_PF_NACC; ++a) sum2 = fadd2(sum2, sum2v[a]);
         float sa, sb;
         f2unpack(sum2, sa, sb);
         l_run += mine ? ((sa + sb) + (suma + sumb)) : 0.f;
