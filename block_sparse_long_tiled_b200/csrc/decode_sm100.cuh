@@ -173,7 +173,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
   const int hs = sub / LPH;             // head whose score this lane holds
   const bool owner = (sub % LPH) == 0;  // one writer per (key, head)
   const int hv = lane % G;              // head this lane votes / keeps state for
-  float qreg[G][PPL * 8];
+  // q as fp32 pairs: the dot products run as packed f32x2 FMAs.
+  uint64_t qreg[G][PPL * 4];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
@@ -182,18 +183,18 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       float f[8];
       bf16x8_to_f32(w, f);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) qreg[g][i * 8 + e] = f[e];
+      for (int e = 0; e < 4; ++e) qreg[g][i * 4 + e] = f2pack(f[2 * e], f[2 * e + 1]);
     }
 
   const bool t_positive = p.tsf > 0.f;
   const float log2_t = t_positive ? (float)log2((double)p.tsf / (double)Lb) : -INFINITY;
   float m_run = -INFINITY;  // running max of head hv (identical in every warp)
   float l_lane = 0.f;       // this lane's share of the row sum of head hs
-  float oacc[G][EPL];
+  uint64_t oacc[G][EPL / 2];  // fp32 pairs of this lane's output columns
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) oacc[g][e] = 0.f;
+    for (int e = 0; e < EPL / 2; ++e) oacc[g][e] = f2pack(0.f, 0.f);
   uint32_t v_phase = 0;      // one parity bit per V slot
   uint64_t kept_mask = 0;    // bit (t % 64): tile t was kept
   int n_skipped = 0;
@@ -211,9 +212,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
 #pragma unroll
       for (int ps = 0; ps < 2; ++ps) {
         const int key = ps * 32 + warp * 4 + kq;
-        float acc[G];
+        uint64_t acc2[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) acc[g] = 0.f;
+        for (int g = 0; g < G; ++g) acc2[g] = f2pack(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < PPL; ++i) {
           const uint4 w =
@@ -221,9 +222,18 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
           float f[8];
           bf16x8_to_f32(w, f);
 #pragma unroll
-          for (int g = 0; g < G; ++g)
+          for (int e = 0; e < 4; ++e) {
+            const uint64_t k2 = f2pack(f[2 * e], f[2 * e + 1]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[g] = fmaf(qreg[g][i * 8 + e], f[e], acc[g]);
+            for (int g = 0; g < G; ++g) acc2[g] = ffma2(qreg[g][i * 4 + e], k2, acc2[g]);
+          }
+        }
+        float acc[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float lo, hi;
+          f2unpack(acc2[g], lo, hi);
+          acc[g] = lo + hi;
         }
         const float dot = transpose_reduce8<G>(acc, sub);
         s[ps] = (key < keys) ? dot * p.scale_log2 : -INFINITY;
@@ -283,8 +293,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float a = Abuf[(u % kDecNPB) * G + g];
+        const uint64_t a2 = f2pack(a, a);
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) oacc[g][e] *= a;
+        for (int e = 0; e < EPL / 2; ++e) oacc[g][e] = fmul2(oacc[g][e], a2);
       }
 #pragma unroll
       for (int k = 0; k < kDecKeysPerWarp; ++k) {
@@ -302,11 +313,15 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
             vf[0] = __uint_as_float(w << 16);
             vf[1] = __uint_as_float(w & 0xFFFF0000u);
           }
+          uint64_t v2[EPL / 2];
+#pragma unroll
+          for (int e = 0; e < EPL / 2; ++e) v2[e] = f2pack(vf[2 * e], vf[2 * e + 1]);
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             const float pk = Pu[k * G + g];
+            const uint64_t p2 = f2pack(pk, pk);
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) oacc[g][e] = fmaf(pk, vf[e], oacc[g][e]);
+            for (int e = 0; e < EPL / 2; ++e) oacc[g][e] = ffma2(p2, v2[e], oacc[g][e]);
           }
         }
       }
@@ -323,7 +338,12 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) red[(warp * G + g) * D + lane * EPL + e] = oacc[g][e];
+    for (int e = 0; e < EPL / 2; ++e) {
+      float lo, hi;
+      f2unpack(oacc[g][e], lo, hi);
+      red[(warp * G + g) * D + lane * EPL + 2 * e] = lo;
+      red[(warp * G + g) * D + lane * EPL + 2 * e + 1] = hi;
+    }
   if (kq == 0 && owner) lsum[warp * G + hs] = lw;
   if (tid == 0 && p.counts) {
     atomicAdd(&p.counts[0], (unsigned long long)n_skipped);
