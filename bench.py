@@ -256,8 +256,7 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     def barrier():
         if world > 1:
@@ -273,86 +272,92 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(
             torch.bfloat16)
 
-    # ---- inputs (host-generated, seeded), resident in HBM before timing
     readings = [r for r in args.readings.split(",") if r]
     if args.reading not in readings:
         readings.insert(0, args.reading)
-    if args.only == "decode":
-        readings = []
-    pre = {}
-    for rd in readings:
-        x = synth.prefill_inputs(w, rd)
-        d = {"q": to_dev(x["q"]), "k": to_dev(x["k"]), "v": to_dev(x["v"])}
-        d["o"] = torch.empty_like(d["q"])
-        d["lse"] = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
-        d["cnt"] = torch.zeros(2, dtype=torch.int64, device=dev)
-        d["host"] = x
-        pre[rd] = d
     dw = decode_workload(args)
-    with_dec = args.only != "prefill"
-    dx = synth.decode_inputs(dw, args.reading) if with_dec else None
-    dec = {} if not with_dec else {
-           "q": to_dev(dx["q"]), "kc": to_dev(dx["kcache"]), "vc": to_dev(dx["vcache"]),
-           "lens": torch.from_numpy(dx["seqlens"]).to(dev),
-           "o": torch.empty((dw.B, dw.Hq, dw.d), dtype=torch.bfloat16, device=dev),
-           "lse": torch.empty((dw.B, dw.Hq), dtype=torch.float32, device=dev),
-           "ws": torch.empty(sk.sskip_attn_decode_workspace_size(dw.B, dw.Hq, dw.d,
-                                                                 dw.num_splits),
-                             dtype=torch.uint8, device=dev),
-           "cnt": torch.zeros(2, dtype=torch.int64, device=dev)}
 
-    def run_prefill(d):
-        sk.sskip_attn_prefill(d["q"], d["k"], d["v"], d["o"], d["lse"], causal=w.causal,
-                              sm_scale=w.scale, threshold_scale_factor=w.tsf, Br=w.Br, Bc=w.Bc,
-                              skip_count=d["cnt"], stream=stream)
+    # ---- legs of the step: prefill and decode, one per generator reading.
+    legs = []
+    if args.only != "decode":
+        for rd in readings:
+            x = synth.prefill_inputs(w, rd)
+            t = {"q": to_dev(x["q"]), "k": to_dev(x["k"]), "v": to_dev(x["v"])}
+            t["o"] = torch.empty_like(t["q"])
+            t["lse"] = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
+            t["cnt"] = torch.zeros(2, dtype=torch.int64, device=dev)
 
-    def run_decode():
-        sk.sskip_attn_decode(dec["q"], dec["kc"], dec["vc"], dec["lens"], dec["o"], dec["lse"],
-                             sm_scale=dw.scale, threshold_scale_factor=dw.tsf, Bc=dw.Bc,
-                             num_splits=dw.num_splits, workspace=dec["ws"],
-                             skip_count=dec["cnt"], stream=stream)
+            def run(t=t, tsf=None, tiles=None):
+                sk.sskip_attn_prefill(t["q"], t["k"], t["v"], t["o"], t["lse"], causal=w.causal,
+                                      sm_scale=w.scale,
+                                      threshold_scale_factor=w.tsf if tsf is None else tsf,
+                                      Br=w.Br, Bc=w.Bc, skip_count=t["cnt"], tile_state=tiles,
+                                      stream=stream)
+            legs.append({"name": f"prefill_{rd}", "kind": "prefill", "reading": rd, "t": t,
+                         "host": x, "run": run, "launches": 1})
+    if args.only != "prefill":
+        for rd in (readings if args.decode_readings == "all" else [args.reading]):
+            dx = synth.decode_inputs(dw, rd)
+            t = {"q": to_dev(dx["q"]), "kc": to_dev(dx["kcache"]), "vc": to_dev(dx["vcache"]),
+                 "lens": torch.from_numpy(dx["seqlens"]).to(dev),
+                 "o": torch.empty((dw.B, dw.Hq, dw.d), dtype=torch.bfloat16, device=dev),
+                 "lse": torch.empty((dw.B, dw.Hq), dtype=torch.float32, device=dev),
+                 "ws": torch.empty(sk.sskip_attn_decode_workspace_size(dw.B, dw.Hq, dw.d,
+                                                                       dw.num_splits),
+                                   dtype=torch.uint8, device=dev),
+                 "cnt": torch.zeros(2, dtype=torch.int64, device=dev)}
 
-    # ---- one untimed pass with tile records: skip counts and V bytes moved
-    stats = {}
-    for rd, d in pre.items():
-        tiles = torch.empty((w.B, w.Hq, w.n_q, w.n_k), dtype=torch.uint8, device=dev)
-        sk.sskip_attn_prefill(d["q"], d["k"], d["v"], d["o"], d["lse"], causal=w.causal,
-                              sm_scale=w.scale, threshold_scale_factor=w.tsf, Br=w.Br, Bc=w.Bc,
-                              skip_count=d["cnt"], tile_state=tiles, stream=stream)
-        c = d["cnt"].cpu().tolist()
-        stats[rd] = {"skipped": c[0], "visited": c[1], **prefill_flops(w, c[1], c[0])}
-    dc, dbytes = None, None
-    if with_dec:
-        dtiles = torch.empty((dw.B, dw.Hkv, -(-dw.Lmax // dw.Bc)), dtype=torch.uint8, device=dev)
-        sk.sskip_attn_decode(dec["q"], dec["kc"], dec["vc"], dec["lens"], dec["o"], dec["lse"],
-                             sm_scale=dw.scale, threshold_scale_factor=dw.tsf, Bc=dw.Bc,
-                             num_splits=dw.num_splits, workspace=dec["ws"],
-                             skip_count=dec["cnt"], tile_state=dtiles, stream=stream)
-        dc = dec["cnt"].cpu().tolist()
-        dbytes = decode_bytes(dw, dx["seqlens"], dtiles.cpu().numpy())
+            def run(t=t, tsf=None, tiles=None):
+                sk.sskip_attn_decode(t["q"], t["kc"], t["vc"], t["lens"], t["o"], t["lse"],
+                                     sm_scale=dw.scale,
+                                     threshold_scale_factor=dw.tsf if tsf is None else tsf,
+                                     Bc=dw.Bc, num_splits=dw.num_splits, workspace=t["ws"],
+                                     skip_count=t["cnt"], tile_state=tiles, stream=stream)
+            legs.append({"name": f"decode_{rd}", "kind": "decode", "reading": rd, "t": t,
+                         "host": {"q": dx["q"], "seqlens": dx["seqlens"]}, "run": run,
+                         "launches": 2})
+            del dx
+
+    # ---- one untimed pass with tile records: skip counts, FLOPs, bytes moved
+    for leg in legs:
+        t = leg["t"]
+        if leg["kind"] == "prefill":
+            tiles = torch.empty((w.B, w.Hq, w.n_q, w.n_k), dtype=torch.uint8, device=dev)
+            leg["run"](tiles=tiles)
+            c = t["cnt"].cpu().tolist()
+            leg["stats"] = {"skipped": c[0], "visited": c[1], **prefill_flops(w, c[1], c[0])}
+        else:
+            tiles = torch.empty((dw.B, dw.Hkv, -(-dw.Lmax // dw.Bc)), dtype=torch.uint8, device=dev)
+            leg["run"](tiles=tiles)
+            c = t["cnt"].cpu().tolist()
+            leg["stats"] = {"skipped": c[0], "visited": c[1],
+                            **decode_bytes(dw, leg["host"]["seqlens"], tiles.cpu().numpy())}
     assert sk.sskip_get_status() == sk.SSKIP_OK
-
-    seg = list(pre) + (["dec"] if with_dec else [])
-    launches_per_step = len(pre) + (2 if with_dec else 0)  # prefill per reading, split + merge
-
-    def step(ev):
-        for rd, d in pre.items():
-            flush.zero_()
-            ev[rd][0].record(stream)
-            run_prefill(d)
-            ev[rd][1].record(stream)
-        if with_dec:
-            flush.zero_()
-            ev["dec"][0].record(stream)
-            run_decode()
-            ev["dec"][1].record(stream)
+    names = [leg["name"] for leg in legs]
 
     def new_events():
-        return {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for k in seg}
+        return {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for n in names}
 
-    for _ in range(args.warmup):
-        step(new_events())
+    def timed(body, steps):
+        """Run `body(events)` steps times after warm-up; device ms per leg, max over ranks."""
+        for _ in range(args.warmup):
+            body(new_events())
+        barrier()
+        evs = [new_events() for _ in range(steps)]
+        for i in range(steps):
+            body(evs[i])
+        barrier()
+        ms = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in evs) / steps for n in names}
+        return dict(zip(names, reduce_max([ms[n] for n in names], world, dev)))
+
+    def step(ev, tsf=None):
+        for leg in legs:
+            flush.zero_()
+            ev[leg["name"]][0].record(stream)
+            leg["run"](tsf=tsf)
+            ev[leg["name"]][1].record(stream)
+
     props = torch.cuda.get_device_properties(dev)
     gpu_id = None
     if getattr(props, "uuid", None) is not None:
@@ -360,148 +365,132 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
         gpu_id = u if u.startswith("GPU-") else f"GPU-{u}"
     clocks = ClockSampler(gpu_id)
     clocks.start()
-    barrier()
-    evs = [new_events() for _ in range(args.steps)]
-    for i in range(args.steps):
-        step(evs[i])
-    barrier()
+    ms = timed(step, args.steps)
     clock_rec = clocks.stop()
     assert sk.sskip_get_status() == sk.SSKIP_OK
 
-    ms = {k: sum(e[k][0].elapsed_time(e[k][1]) for e in evs) for k in seg}
-    keys = list(ms)
-    ms = dict(zip(keys, reduce_max([ms[k] for k in keys], world, dev)))
-    K = args.steps
+    # ---- skip-disabled control: the same kernels and inputs at tsf = 0
+    ms_dense = timed(lambda ev: step(ev, tsf=0.0), max(3, args.steps // 3)) \
+        if not args.no_control else {}
 
-    if args.no_e2e:
-        ems, hp, ho, hq_dec, hl_dec, ho_dec = None, {}, {}, None, None, None
-    else:
-        ems, hp, ho, hq_dec, hl_dec, ho_dec = time_e2e(args, pre, dec, dx, with_dec, seg, keys,
-                                                      run_prefill, run_decode, flush, stream,
-                                                      new_events, barrier, world, dev, K)
+    # ---- end to end through the public API: pinned host in, host out
+    ems, io_bytes = ({}, (0, 0)) if args.no_e2e else time_e2e(legs, flush, stream, new_events,
+                                                             timed, args.steps)
+
     if rank == 0:
-        print(json.dumps(report(args, w, world, pre, stats, ms, ems, K, peaks, peak_kind, dw, dbytes,
-                                dc, hp, ho, hq_dec, hl_dec, ho_dec, clock_rec,
-                                launches_per_step)), flush=True)
+        print(json.dumps(report(args, w, dw, world, legs, ms, ms_dense, ems, io_bytes, peaks,
+                                peak_kind, clock_rec)), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
 
 
-def time_e2e(args, pre, dec, dx, with_dec, seg, keys, run_prefill, run_decode, flush, stream,
-             new_events, barrier, world, dev, K):
-    """Same steps through the public API with pinned host buffers: H2D of the
-    step's inputs and D2H of its outputs inside the timed region."""
+def time_e2e(legs, flush, stream, new_events, timed, steps):
+    """Same steps with each leg's inputs copied host->device from pinned memory
+    and its outputs copied back inside the timed region."""
     import torch
-    hp = {rd: {n: torch.from_numpy(np.ascontiguousarray(pre[rd]["host"][n]).view(np.int16))
-               .view(torch.bfloat16).pin_memory() for n in ("q", "k", "v")} for rd in pre}
-    ho = {rd: (torch.empty_like(pre[rd]["o"], device="cpu").pin_memory(),
-               torch.empty_like(pre[rd]["lse"], device="cpu").pin_memory()) for rd in pre}
-    hq_dec = hl_dec = ho_dec = None
-    if with_dec:
-        hq_dec = torch.from_numpy(np.ascontiguousarray(dx["q"]).view(np.int16)).view(
-            torch.bfloat16).pin_memory()
-        hl_dec = torch.from_numpy(dx["seqlens"]).pin_memory()
-        ho_dec = (torch.empty_like(dec["o"], device="cpu").pin_memory(),
-                  torch.empty_like(dec["lse"], device="cpu").pin_memory())
+    h2d = d2h = 0
+    for leg in legs:
+        t = leg["t"]
+        if leg["kind"] == "prefill":
+            leg["pin_in"] = {n: torch.from_numpy(np.ascontiguousarray(leg["host"][n]).view(
+                np.int16)).view(torch.bfloat16).pin_memory() for n in ("q", "k", "v")}
+            leg["dev_in"] = {n: t[n] for n in ("q", "k", "v")}
+        else:
+            leg["pin_in"] = {"q": torch.from_numpy(np.ascontiguousarray(leg["host"]["q"]).view(
+                np.int16)).view(torch.bfloat16).pin_memory(),
+                "lens": torch.from_numpy(leg["host"]["seqlens"]).pin_memory()}
+            leg["dev_in"] = {"q": t["q"], "lens": t["lens"]}
+        leg["pin_out"] = (torch.empty_like(t["o"], device="cpu").pin_memory(),
+                          torch.empty_like(t["lse"], device="cpu").pin_memory())
+        h2d += sum(int(v.numel() * v.element_size()) for v in leg["pin_in"].values())
+        d2h += sum(int(v.numel() * v.element_size()) for v in leg["pin_out"])
 
     def e2e_step(ev):
-        for rd, d in pre.items():
+        for leg in legs:
+            t = leg["t"]
             flush.zero_()
-            ev[rd][0].record(stream)
-            for n in ("q", "k", "v"):
-                d[n].copy_(hp[rd][n], non_blocking=True)
-            run_prefill(d)
-            ho[rd][0].copy_(d["o"], non_blocking=True)
-            ho[rd][1].copy_(d["lse"], non_blocking=True)
-            ev[rd][1].record(stream)
-        if with_dec:
-            flush.zero_()
-            ev["dec"][0].record(stream)
-            dec["q"].copy_(hq_dec, non_blocking=True)
-            dec["lens"].copy_(hl_dec, non_blocking=True)
-            run_decode()
-            ho_dec[0].copy_(dec["o"], non_blocking=True)
-            ho_dec[1].copy_(dec["lse"], non_blocking=True)
-            ev["dec"][1].record(stream)
+            ev[leg["name"]][0].record(stream)
+            for n, hv in leg["pin_in"].items():
+                leg["dev_in"][n].copy_(hv, non_blocking=True)
+            leg["run"]()
+            leg["pin_out"][0].copy_(t["o"], non_blocking=True)
+            leg["pin_out"][1].copy_(t["lse"], non_blocking=True)
+            ev[leg["name"]][1].record(stream)
 
-    for _ in range(args.warmup):
-        e2e_step(new_events())
-    barrier()
-    eevs = [new_events() for _ in range(K)]
-    for i in range(K):
-        e2e_step(eevs[i])
-    barrier()
-    ems = {k: sum(e[k][0].elapsed_time(e[k][1]) for e in eevs) for k in keys}
-    ems = dict(zip(keys, reduce_max([ems[k] for k in keys], world, dev)))
-    return ems, hp, ho, hq_dec, hl_dec, ho_dec
+    return timed(e2e_step, steps), (h2d, d2h)
 
 
-def report(args, w, world, pre, stats, ms, ems, K, peaks, peak_kind, dw, dbytes, dc, hp, ho,
-           hq_dec, hl_dec, ho_dec, clock_rec, launches_per_step) -> dict:
-    head = args.reading
+def report(args, w, dw, world, legs, ms, ms_dense, ems, io_bytes, peaks, peak_kind,
+           clock_rec) -> dict:
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    K = args.steps
     line = {"metric": METRIC, "value": None, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
-            "warmup": args.warmup, "ms_per_step": sum(ms.values()) / K,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": config_block(w, args)}
-
-    def prefill_block(rd):
-        s = stats[rd]
-        t = ms[rd] / K / 1e3
-        b = {"ms_per_launch": t * 1e3, "executed_tflops": s["executed"] / t / 1e12,
-             "dense_equiv_tflops": s["dense"] / t / 1e12,
-             "executed_frac_of_peak": s["executed"] / t / 1e12 / peak,
-             "skip_fraction": s["skipped"] / max(1, s["visited"]),
-             "skipped_tiles": s["skipped"], "visited_tiles": s["visited"],
-             "executed_tflop": s["executed"] / 1e12, "dense_equiv_tflop": s["dense"] / 1e12}
-        if ems is not None:
-            b["e2e_ms_per_step"] = ems[rd] / K
-        return b
-
+            "warmup": args.warmup, "ms_per_step": sum(ms.values()), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_block(w, args)}
+    pre, dec = {}, {}
+    for leg in legs:
+        n, s = leg["name"], leg["stats"]
+        t = ms[n] / 1e3
+        b = {"ms_per_launch": ms[n], "skip_fraction": s["skipped"] / max(1, s["visited"]),
+             "skipped_tiles": s["skipped"], "visited_tiles": s["visited"]}
+        if leg["kind"] == "prefill":
+            b.update(executed_tflops=s["executed"] / t / 1e12,
+                     dense_equiv_tflops=s["dense"] / t / 1e12,
+                     executed_frac_of_peak=s["executed"] / t / 1e12 / peak,
+                     executed_tflop=s["executed"] / 1e12, dense_equiv_tflop=s["dense"] / 1e12)
+            ideal = 1.0 / (1.0 - b["skip_fraction"] / 2.0)
+        else:
+            b.update(gbs_actually_moved=s["total"] / t / 1e9,
+                     frac_of_hbm=s["total"] / t / 1e9 / hbm,
+                     bytes_actually_moved=s["total"], bytes_if_no_skip=s["total_dense"])
+            ideal = s["total_dense"] / s["total"]
+        if n in ms_dense:
+            b.update(ms_skip_disabled=ms_dense[n], speedup_vs_skip_disabled=ms_dense[n] / ms[n],
+                     ideal_speedup=ideal)
+        if n in ems:
+            b["e2e_ms"] = ems[n]
+        (pre if leg["kind"] == "prefill" else dec)[leg["reading"]] = b
+    head = args.reading
     if pre:
-        st = stats[head]
-        t_launch = ms[head] / K / 1e3  # seconds per prefill launch
-        achieved = st["executed"] / t_launch / 1e12
-        line["value"] = world * st["executed"] * K / (ms[head] / 1e3) / 1e12
+        hs = next(leg["stats"] for leg in legs if leg["name"] == f"prefill_{head}")
+        t = ms[f"prefill_{head}"] / 1e3
+        achieved = hs["executed"] / t / 1e12
+        line["value"] = world * achieved
         line["roofline"] = {
             "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": ncu_traffic("prefill_kernel"),
             "kernel": f"prefill_kernel<{w.d},{w.Br},{w.Bc},{'causal' if w.causal else 'full'}>",
             "peak_source": f"{peak_kind} bf16_tflops (burst; kernel timed alone)"}
-        line["prefill"] = {rd: prefill_block(rd) for rd in pre}
-    if dbytes is not None:
-        t_dec = ms["dec"] / K / 1e3
-        dec_gbs = dbytes["total"] / t_dec / 1e9
-        line["decode"] = {
-            "workload": dw.name, "ms_per_launch": t_dec * 1e3, "gbs_actually_moved": dec_gbs,
-            "frac_of_hbm": dec_gbs / hbm, "hbm_peak_gbs": hbm,
-            "bytes_actually_moved": dbytes["total"], "bytes_if_no_skip": dbytes["total_dense"],
-            "skip_fraction": dc[0] / max(1, dc[1]), "skipped_tiles": dc[0],
-            "visited_tiles": dc[1],
-            "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm, "unit": "GB/s",
-                         "frac": dec_gbs / hbm, "traffic": ncu_traffic("decode_split_kernel"),
-                         "peak_source": f"{peak_kind} hbm_gbs"}}
-        if ems is not None:
-            line["decode"]["e2e_ms_per_step"] = ems["dec"] / K
+        line["prefill"] = pre
+        if ems:
+            line["e2e"] = {"value": world * hs["executed"] / (ems[f"prefill_{head}"] / 1e3) / 1e12,
+                           "unit": "TFLOP/s", "h2d_bytes_per_step": io_bytes[0],
+                           "d2h_bytes_per_step": io_bytes[1]}
+    if dec:
+        dkey = head if head in dec else next(iter(dec))
+        dstats = next(leg["stats"] for leg in legs if leg["name"] == f"decode_{dkey}")
+        gbs = dec[dkey]["gbs_actually_moved"]
+        dec["workload"] = dw.name
+        dec["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                           "frac": gbs / hbm, "traffic": ncu_traffic("decode_split_kernel"),
+                           "reading": dkey, "peak_source": f"{peak_kind} hbm_gbs"}
+        line["decode"] = dec
         if not pre:  # decode-only runs report GB/s as the value
-            line.update(value=world * dec_gbs, unit="GB/s", roofline=line["decode"]["roofline"])
-    if ems is not None and pre:
-        h2d = sum(int(t.numel() * t.element_size()) for rd in pre for t in hp[rd].values())
-        d2h = sum(int(a.numel() * a.element_size() + b.numel() * b.element_size())
-                  for a, b in ho.values())
-        if hq_dec is not None:
-            h2d += int(hq_dec.numel() * 2 + hl_dec.numel() * 4)
-            d2h += int(ho_dec[0].numel() * 2 + ho_dec[1].numel() * 4)
-        line["e2e"] = {"value": world * stats[head]["executed"] * K / (ems[head] / 1e3) / 1e12,
-                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            line.update(value=world * gbs, unit="GB/s", roofline=dec["roofline"])
+            if ems:
+                line["e2e"] = {"value": world * dstats["total"] / (ems[f"decode_{dkey}"] / 1e3) / 1e9,
+                               "unit": "GB/s", "h2d_bytes_per_step": io_bytes[0],
+                               "d2h_bytes_per_step": io_bytes[1]}
     line["clocks"] = clock_rec
-    line["gpu_launches"] = launches_per_step * K
+    line["gpu_launches"] = sum(leg["launches"] for leg in legs) * K
     if not args.no_cpu_baseline and world == 1 and pre:
         units = oracle_sample_units(w, heads=args.cpu_heads)
         threads = os.cpu_count() or 1
-        r = time_oracle(w, pre[head]["host"], units, threads)
+        hx = next(leg["host"] for leg in legs if leg["name"] == f"prefill_{head}")
+        r = time_oracle(w, hx, units, threads)
         line["cpu_baseline"] = {
             "value": r["executed_flops"] / r["seconds"] / 1e12, "unit": "TFLOP/s",
             "cores": threads, "kind": "oracle", "seconds": r["seconds"],
@@ -509,6 +498,54 @@ def report(args, w, world, pre, stats, ms, ems, K, peaks, peak_kind, dw, dbytes,
                        f"({args.cpu_heads / w.Hq:.3f} of {w.name}, {head} reading), "
                        f"executed FLOPs / wall time")}
     return line
+
+
+def run_sweep(args):
+    """Long-prefill threshold sweep: speed vs skip fraction at each factor."""
+    import torch
+    import block_sparse_long_tiled_b200 as sk
+    dev = torch.device("cuda", 0)
+    peaks, _ = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    w0 = synth.PREFILL_WORKLOADS[args.prefill]
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for rd in [r for r in args.readings.split(",") if r]:
+        x = synth.prefill_inputs(w0, rd)
+        td = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev).view(
+            torch.bfloat16)
+        q, k, v = td(x["q"]), td(x["k"]), td(x["v"])
+        del x
+        base_ms = None
+        for tsf in synth.LLAMA70B_TSF_SWEEP:
+            w = w0.replace(tsf=tsf)
+            out = sk.prefill(q, k, v, causal=w.causal, sm_scale=w.scale,
+                             threshold_scale_factor=tsf, Br=w.Br, Bc=w.Bc)
+            c = out["counts"].cpu().tolist()
+            ts = []
+            for i in range(args.warmup + args.steps):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                sk.sskip_attn_prefill(q, k, v, out["o"], out["lse"], causal=w.causal,
+                                      sm_scale=w.scale, threshold_scale_factor=tsf, Br=w.Br,
+                                      Bc=w.Bc)
+                b.record()
+                torch.cuda.synchronize()
+                if i >= args.warmup:
+                    ts.append(a.elapsed_time(b))
+            ms = float(np.median(ts))
+            base_ms = ms if tsf == 0 else base_ms
+            f = prefill_flops(w, c[1], c[0])
+            s = c[0] / max(1, c[1])
+            print(json.dumps({"sweep": w.name, "reading": rd, "threshold_scale_factor": tsf,
+                              "ms": ms, "skip_fraction": s,
+                              "executed_tflops": f["executed"] / ms / 1e9,
+                              "executed_frac_of_peak": f["executed"] / ms / 1e9 / peak,
+                              "dense_equiv_tflops": f["dense"] / ms / 1e9,
+                              "speedup_vs_tsf0": (base_ms / ms) if base_ms else None,
+                              "ideal_speedup": 1.0 / (1.0 - s / 2.0)}), flush=True)
+        del q, k, v
+        torch.cuda.empty_cache()
 
 
 def decode_workload(args):
@@ -538,6 +575,11 @@ def main(argv=None):
     ap.add_argument("--cpu-heads", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-control", action="store_true",
+                    help="skip the tsf = 0 (skipping disabled) control timing")
+    ap.add_argument("--decode-readings", choices=["all", "headline"], default="all")
+    ap.add_argument("--sweep", action="store_true",
+                    help="threshold sweep of --prefill (default: the 128K long prefill)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
@@ -549,6 +591,9 @@ def main(argv=None):
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE {world}")
     if args.impl == "reference":
         run_reference(args, w, rank)
+        return
+    if args.sweep:
+        run_sweep(args)
         return
     run_gpu(args, w, rank, world, local_rank)
 
