@@ -52,7 +52,7 @@ def _load():
         for suf in ("_f32", "_f64"):
             f = getattr(lib, "sskip_oracle_prefill" + suf)
             f.restype = I
-            f.argtypes = [P, P, P, I, I, I, I, I, I, D, D, I, I, P, I, P, P, P, P, P, I]
+            f.argtypes = [P, P, P, I, I, I, I, I, I, D, D, I, I, I, P, I, P, P, P, P, P, P, I]
             g = getattr(lib, "sskip_oracle_decode" + suf)
             g.restype = I
             g.argtypes = [P, P, P, P, I, I, I, I, I, D, D, I, I, P, P, P, P, P, P, P, I]
@@ -77,13 +77,19 @@ def default_threads() -> int:
 
 def prefill(q, k, v, *, causal: bool, sm_scale: float, tsf: float, Br: int, Bc: int,
             units=None, precision: str = "f32", nthreads: int | None = None,
-            want_margin: bool = False) -> dict:
+            want_margin: bool = False, vote_rows: int | None = None) -> dict:
     """Skip-Softmax prefill on bf16 bits q [B,Hq,L,d], k/v [B,Hkv,L,d].
 
     ``units``: optional int array of (b, hq, i) query-tile units; when given,
     outputs are per unit: o [n,Br,d], lse [n,Br], tile_state [n,n_k].
     Otherwise o [B,Hq,L,d], lse [B,Hq,L], tile_state [B,Hq,n_q,n_k].
     tile_state: 0 = not visited, 1 = kept, 2 = skipped.
+
+    ``vote_rows``: rows per vote (default Br, the block vote). A smaller
+    divisor of Br cuts each query tile into slices that vote alone (the
+    warp-granular variant); ``slice_mask`` then records per tile 0 (not
+    visited) or 0x80 | the bitmask of slices that skipped it, and
+    ``slices_skipped`` / ``slices_visited`` count slices holding a valid row.
     """
     q, k, v = _u16(q), _u16(k), _u16(v)
     B, Hq, L, d = q.shape
@@ -99,24 +105,28 @@ def prefill(q, k, v, *, causal: bool, sm_scale: float, tsf: float, Br: int, Bc: 
         n = B * Hq * n_q
     o = np.empty((n, Br, d), real)
     lse = np.empty((n, Br), real)
-    counts = np.zeros(2, np.int64)
+    counts = np.zeros(4, np.int64)
     state = np.empty((n, n_k), np.int8)
+    smask = np.empty((n, n_k), np.uint8)
     margin = np.empty((n, n_k), real) if want_margin else None
     fn = getattr(_load(), "sskip_oracle_prefill_" + precision)
     rc = fn(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, L, d, int(causal), float(sm_scale),
-            float(tsf), Br, Bc, _ptr(units), n, _ptr(o), _ptr(lse), _ptr(counts),
-            _ptr(state), _ptr(margin), int(nthreads or default_threads()))
+            float(tsf), Br, Bc, int(Br if vote_rows is None else vote_rows), _ptr(units), n, _ptr(o), _ptr(lse),
+            _ptr(counts), _ptr(state), _ptr(smask), _ptr(margin),
+            int(nthreads or default_threads()))
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
-    out = {"skipped": int(counts[0]), "visited": int(counts[1])}
+    out = {"skipped": int(counts[0]), "visited": int(counts[1]),
+           "slices_skipped": int(counts[2]), "slices_visited": int(counts[3])}
     if units is None:
         out["o"] = o.reshape(B, Hq, n_q * Br, d)[:, :, :L]
         out["lse"] = lse.reshape(B, Hq, n_q * Br)[:, :, :L]
         out["tile_state"] = state.reshape(B, Hq, n_q, n_k)
+        out["slice_mask"] = smask.reshape(B, Hq, n_q, n_k)
         if margin is not None:
             out["tile_margin"] = margin.reshape(B, Hq, n_q, n_k)
     else:
-        out.update(o=o, lse=lse, tile_state=state)
+        out.update(o=o, lse=lse, tile_state=state, slice_mask=smask)
         if margin is not None:
             out["tile_margin"] = margin
     return out

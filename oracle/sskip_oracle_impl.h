@@ -22,6 +22,12 @@
  *     and finite m_local fails;
  *   - a block is skipped only when every valid row passes; padding rows
  *     (index >= L) do not vote;
+ *   - optional finer vote (SpargeAttn article, "稀疏 Warp 在线 Softmax"
+ *     stage: the same local-vs-global maximum test taken per warp): the Br
+ *     rows of a query tile are cut into slices of vote_rows rows, each
+ *     slice votes alone with the same rule and a slice that passes leaves
+ *     its rows' m, l and O untouched; the block (its V and P.V) is skipped
+ *     only when every slice passes.  vote_rows = Br is the block vote;
  *   - key blocks are visited in ascending order; m_run is the state before
  *     the block; a skipped block leaves m, l and O untouched;
  *   - prefill: a block is Br rows of ONE query head; query head hq reads kv
@@ -65,23 +71,25 @@ static REAL FN(dot)(const REAL* a, const REAL* b, int d) {
 /* ------------------------------------------------------------------ */
 typedef struct {
     const uint16_t *q, *k, *v;
-    int B, Hq, Hkv, L, d, causal, Br, Bc;
+    int B, Hq, Hkv, L, d, causal, Br, Bc, vote_rows;
     REAL scale, ln_t;
     int t_positive;
     const int32_t* units; /* (b, hq, i) triples or NULL = natural order */
     int n_units;
     REAL *o, *lse;        /* [n_units][Br][d], [n_units][Br] */
     int8_t* tile_state;   /* [n_units][n_k] or NULL */
+    uint8_t* slice_mask;  /* [n_units][n_k] or NULL: 0 unvisited, else 0x80 | skipped slices */
     REAL* tile_margin;    /* [n_units][n_k] or NULL */
-    int64_t skipped, visited;
+    int64_t skipped, visited, sl_skipped, sl_visited;
     int next;             /* work counter */
     pthread_mutex_t mu;
 } FN(prefill_job);
 
 static void FN(prefill_unit)(FN(prefill_job)* J, int u, REAL* qf, REAL* kf, REAL* vf,
                              REAL* S, REAL* m_run, REAL* l, REAL* m_loc,
-                             int64_t* skipped, int64_t* visited) {
+                             int64_t* cnt /* skipped, visited, slices skipped, slices visited */) {
     const int d = J->d, Br = J->Br, Bc = J->Bc, L = J->L;
+    const int R = J->vote_rows, n_sl = Br / R;
     const int n_q = (L + Br - 1) / Br, n_k = (L + Bc - 1) / Bc;
     int b, hq, i;
     if (J->units) {
@@ -109,6 +117,8 @@ static void FN(prefill_unit)(FN(prefill_job)* J, int u, REAL* qf, REAL* kf, REAL
     }
     if (J->tile_state)
         for (int j = 0; j < n_k; ++j) J->tile_state[(size_t)u * n_k + j] = 0;
+    if (J->slice_mask)
+        for (int j = 0; j < n_k; ++j) J->slice_mask[(size_t)u * n_k + j] = 0;
 
     for (int j = 0; j <= j_max; ++j) {
         const int key0 = j * Bc;
@@ -128,23 +138,34 @@ static void FN(prefill_unit)(FN(prefill_job)* J, int u, REAL* qf, REAL* kf, REAL
             m_loc[r] = mx;
         }
 
-        /* Step 2: compare with the running maximum; every valid row votes. */
+        /* Step 2: compare with the running maximum; every valid row votes,
+         * and each slice of R rows decides for itself.  A slice without a
+         * valid row passes vacuously and is not counted. */
         int skip = 1;
+        unsigned sl_pass = 0;
         REAL margin = (REAL)INFINITY;
-        for (int r = 0; r < rows; ++r) {
-            if (!FN(row_passes)(m_loc[r], m_run[r], J->ln_t, J->t_positive)) skip = 0;
-            REAL mg = FN(row_margin)(m_loc[r], m_run[r], J->ln_t, J->t_positive);
-            if (mg < margin) margin = mg;
+        for (int sl = 0; sl < n_sl; ++sl) {
+            int pass = 1;
+            for (int r = sl * R; r < (sl + 1) * R && r < rows; ++r) {
+                if (!FN(row_passes)(m_loc[r], m_run[r], J->ln_t, J->t_positive)) pass = 0;
+                REAL mg = FN(row_margin)(m_loc[r], m_run[r], J->ln_t, J->t_positive);
+                if (mg < margin) margin = mg;
+            }
+            if (pass) sl_pass |= 1u << sl;
+            else skip = 0;
+            if (sl * R < rows) { cnt[3] += 1; cnt[2] += pass; }
         }
-        *visited += 1;
+        cnt[1] += 1;
         if (J->tile_state) J->tile_state[(size_t)u * n_k + j] = skip ? 2 : 1;
+        if (J->slice_mask) J->slice_mask[(size_t)u * n_k + j] = (uint8_t)(0x80u | sl_pass);
         if (J->tile_margin) J->tile_margin[(size_t)u * n_k + j] = margin;
 
         /* Step 3: a skipped block costs no softmax, no P.V and no V block. */
-        if (skip) { *skipped += 1; continue; }
+        if (skip) { cnt[0] += 1; continue; }
 
         for (int c = 0; c < keys * d; ++c) vf[c] = (REAL)bf16_to_float(vp[(size_t)key0 * d + c]);
         for (int r = 0; r < rows; ++r) {
+            if (sl_pass >> (r / R) & 1u) continue; /* this row's slice skipped the block */
             REAL m_new = m_loc[r] > m_run[r] ? m_loc[r] : m_run[r];
             if (m_new == -(REAL)INFINITY) continue; /* nothing visible yet */
             REAL alpha = (m_run[r] == -(REAL)INFINITY) ? 0 : EXP(m_run[r] - m_new);
@@ -186,15 +207,17 @@ static void* FN(prefill_worker)(void* arg) {
     REAL* m_run = (REAL*)malloc(sizeof(REAL) * Br);
     REAL* l = (REAL*)malloc(sizeof(REAL) * Br);
     REAL* m_loc = (REAL*)malloc(sizeof(REAL) * Br);
-    int64_t skipped = 0, visited = 0;
+    int64_t cnt[4] = {0, 0, 0, 0};
     for (;;) {
         int u = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
         if (u >= J->n_units) break;
-        FN(prefill_unit)(J, u, qf, kf, vf, S, m_run, l, m_loc, &skipped, &visited);
+        FN(prefill_unit)(J, u, qf, kf, vf, S, m_run, l, m_loc, cnt);
     }
     pthread_mutex_lock(&J->mu);
-    J->skipped += skipped;
-    J->visited += visited;
+    J->skipped += cnt[0];
+    J->visited += cnt[1];
+    J->sl_skipped += cnt[2];
+    J->sl_visited += cnt[3];
     pthread_mutex_unlock(&J->mu);
     free(qf); free(kf); free(vf); free(S); free(m_run); free(l); free(m_loc);
     return NULL;
@@ -203,28 +226,34 @@ static void* FN(prefill_worker)(void* arg) {
 int FN(sskip_oracle_prefill)(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                              int B, int Hq, int Hkv, int L, int d, int causal,
                              double sm_scale, double threshold_scale_factor, int Br, int Bc,
-                             const int32_t* units, int n_units,
-                             REAL* o, REAL* lse, int64_t* counts,
-                             int8_t* tile_state, REAL* tile_margin, int nthreads) {
+                             int vote_rows, const int32_t* units, int n_units,
+                             REAL* o, REAL* lse, int64_t* counts /* [4] */,
+                             int8_t* tile_state, uint8_t* slice_mask, REAL* tile_margin,
+                             int nthreads) {
     if (!q || !k || !v || !o || !lse || !counts) return 1;
     if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || L < 1 || d < 1 || Br < 1 || Bc < 1) return 1;
+    if (vote_rows < 1 || vote_rows > Br || Br % vote_rows || Br / vote_rows > 7) return 1;
     if (!(threshold_scale_factor >= 0)) return 1;
     FN(prefill_job) J;
     memset(&J, 0, sizeof(J));
     J.q = q; J.k = k; J.v = v;
     J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.L = L; J.d = d; J.causal = causal; J.Br = Br; J.Bc = Bc;
+    J.vote_rows = vote_rows;
     J.scale = (REAL)sm_scale;
     /* t = threshold_scale_factor / L; compare in the log domain. */
     J.t_positive = threshold_scale_factor > 0;
     J.ln_t = J.t_positive ? (REAL)log(threshold_scale_factor / (double)L) : -(REAL)INFINITY;
     J.units = units;
     J.n_units = units ? n_units : B * Hq * ((L + Br - 1) / Br);
-    J.o = o; J.lse = lse; J.tile_state = tile_state; J.tile_margin = tile_margin;
+    J.o = o; J.lse = lse; J.tile_state = tile_state; J.slice_mask = slice_mask;
+    J.tile_margin = tile_margin;
     pthread_mutex_init(&J.mu, NULL);
     run_workers(FN(prefill_worker), &J, nthreads, J.n_units);
     pthread_mutex_destroy(&J.mu);
     counts[0] = J.skipped;
     counts[1] = J.visited;
+    counts[2] = J.sl_skipped;
+    counts[3] = J.sl_visited;
     return 0;
 }
 

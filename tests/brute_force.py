@@ -154,3 +154,74 @@ def decode_prefix_max_states(q_bits, kc_bits, seqlens, *, scale, tsf, Bc, num_sp
                     states[b, h, j] = 2 if passes.all() else 1
                     prefix = np.maximum(prefix, ml)
     return states
+
+
+def prefix_max_row_passes(q_bits, k_bits, *, causal, scale, tsf, Br, Bc):
+    """Closed-form vote of every row on every tile its query tile visits (t < 1).
+
+    Returns (passes [B,H,L,n_k] bool, visited [n_q,n_k] bool). Same argument as
+    ``prefix_max_states``: while t < 1 no passing block can raise a row's
+    running maximum, so the maximum before block j is the prefix maximum of the
+    row's local maxima over blocks 0..j-1, whatever its slice decided.
+    """
+    S = logits(q_bits, k_bits, scale)
+    B, H, L, _ = S.shape
+    n_q, n_k = -(-L // Br), -(-L // Bc)
+    ln_t = math.log(tsf / L) if tsf > 0 else -math.inf
+    if causal:
+        S = np.where(causal_mask(L), S, -np.inf)
+    m_loc = np.stack([S[..., j * Bc:min(L, (j + 1) * Bc)].max(axis=-1) for j in range(n_k)],
+                     axis=-1)  # [B,H,L,n_k]
+    passes = np.zeros((B, H, L, n_k), bool)
+    visited = np.zeros((n_q, n_k), bool)
+    prefix = np.full((B, H, L), -np.inf)
+    for j in range(n_k):
+        ml = m_loc[..., j]
+        with np.errstate(invalid="ignore"):
+            passes[..., j] = np.where(ml == -np.inf, ln_t > -np.inf,
+                                      np.where(prefix == -np.inf, False, (ml - prefix) < ln_t))
+        prefix = np.maximum(prefix, ml)
+    for i in range(n_q):
+        j_max = min(n_k - 1, ((i + 1) * Br - 1) // Bc) if causal else n_k - 1
+        visited[i, :j_max + 1] = True
+    return passes, visited
+
+
+def slice_masks(passes, visited, *, L, Br, R):
+    """Per (b, h, query tile, key tile): 0 if not visited, else 0x80 | bitmask
+    of the R-row slices whose every valid row passes (a slice with no valid
+    row passes vacuously)."""
+    B, H, _, n_k = passes.shape
+    n_q = visited.shape[0]
+    out = np.zeros((B, H, n_q, n_k), np.uint8)
+    for i in range(n_q):
+        for j in range(n_k):
+            if not visited[i, j]:
+                continue
+            m = 0x80
+            for s in range(Br // R):
+                r0, r1 = i * Br + s * R, min(L, i * Br + (s + 1) * R)
+                m_s = np.ones((B, H), bool) if r0 >= r1 else passes[:, :, r0:r1, j].all(axis=-1)
+                out[:, :, i, j] |= np.where(m_s, 1 << s, 0).astype(np.uint8)
+            out[:, :, i, j] |= m
+    return out
+
+
+def slice_kept_key_mask(slice_mask, L, Br, Bc, R, causal):
+    """slice_mask [B,H,n_q,n_k] -> allowed [B,H,L,L]: row r sees the keys of
+    tile j iff its query tile visited j and r's slice did not skip it."""
+    r = np.arange(L)
+    bit = ((r % Br) // R).astype(np.uint8)
+    sm = slice_mask[:, :, r // Br]                       # [B,H,L,n_k]
+    kept_tile = (sm & 0x80).astype(bool) & ~((sm >> bit[None, None, :, None]) & 1).astype(bool)
+    allowed = kept_tile[..., np.arange(L) // Bc]
+    if causal:
+        allowed = allowed & causal_mask(L)
+    return allowed
+
+
+def slice_restricted_attention(q_bits, k_bits, v_bits, slice_mask, *, causal, scale, Br, Bc, R):
+    S = logits(q_bits, k_bits, scale)
+    L = S.shape[-1]
+    return masked_softmax_attention(S, v_bits,
+                                    slice_kept_key_mask(slice_mask, L, Br, Bc, R, causal))

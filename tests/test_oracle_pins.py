@@ -17,7 +17,8 @@ import pytest
 import oracle
 import synth
 from brute_force import (decode_dense, decode_prefix_max_states, dense_attention,
-                         prefix_max_states, restricted_attention)
+                         prefix_max_row_passes, prefix_max_states, restricted_attention,
+                         slice_masks, slice_restricted_attention)
 from synth import PrefillWorkload, DecodeWorkload, bf16_bits, bf16_to_f32
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -390,3 +391,124 @@ def test_oracle_rejects_bad_arguments():
                        Br=64, Bc=64)
     with pytest.raises(ValueError):
         oracle.prefill(x["q"], x["k"], x["v"], causal=True, sm_scale=1, tsf=-1, Br=64, Bc=64)
+
+
+# --------------------------------------------------------------------------
+# Warp-granular vote (SpargeAttn article, "稀疏 Warp 在线 Softmax" stage:
+# the local-vs-global maximum test per warp): slices of R rows vote alone.
+# --------------------------------------------------------------------------
+SLICE_CASES = [
+    dict(causal=True, L=512, Br=128, Bc=128, tsf=60.0, d=32, R=32),
+    dict(causal=True, L=700, Br=128, Bc=128, tsf=40.0, d=64, R=32, Hq=4, Hkv=2),
+    dict(causal=False, L=333, Br=64, Bc=64, tsf=30.0, R=32, Hq=2, Hkv=1),
+    dict(causal=True, L=448, Br=128, Bc=128, tsf=50.0, d=32, R=64),
+]
+
+
+def _slice_case(kw):
+    kw = dict(kw)
+    R = kw.pop("R")
+    w = small_prefill(**kw)
+    return w, R, synth.prefill_inputs(w, "rms")
+
+
+@pytest.mark.parametrize("kw", SLICE_CASES)
+def test_slice_votes_equal_prefix_max_closed_form(kw):
+    w, R, x = _slice_case(kw)
+    assert w.tsf / w.L < 1
+    got = run_prefill(w, x, "f64", vote_rows=R)
+    passes, visited = prefix_max_row_passes(x["q"], x["k"], causal=w.causal, scale=w.scale,
+                                            tsf=w.tsf, Br=w.Br, Bc=w.Bc)
+    want = slice_masks(passes, visited, L=w.L, Br=w.Br, R=R)
+    np.testing.assert_array_equal(got["slice_mask"], want)
+    # The block decision is the AND of the slices (every slice bit set).
+    full = np.uint8(0x80 | ((1 << (w.Br // R)) - 1))
+    np.testing.assert_array_equal(got["tile_state"] == 2, want == full)
+    # Slices that vote to skip while their block is kept: the variant's gain.
+    assert np.any((want != full) & (want & 0x7F != 0) & (want != 0)), "case must hit partial skips"
+
+
+@pytest.mark.parametrize("precision", ["f32", "f64"])
+@pytest.mark.parametrize("kw", SLICE_CASES)
+def test_slice_vote_output_equals_row_restricted_dense(kw, precision):
+    w, R, x = _slice_case(kw)
+    got = run_prefill(w, x, precision, vote_rows=R)
+    O, lse = slice_restricted_attention(x["q"], x["k"], x["v"], got["slice_mask"],
+                                        causal=w.causal, scale=w.scale, Br=w.Br, Bc=w.Bc, R=R)
+    tol = 3e-5 if precision == "f32" else 1e-11
+    np.testing.assert_allclose(got["o"], O, atol=tol, rtol=0)
+    np.testing.assert_allclose(got["lse"], lse, atol=tol, rtol=0)
+
+
+@pytest.mark.parametrize("kw", SLICE_CASES)
+def test_slice_vote_keeps_block_decisions_and_counts(kw):
+    # While t < 1 a passing row never moves its maximum, so the running maxima
+    # and hence the block decisions are the same under both granularities.
+    w, R, x = _slice_case(kw)
+    blk = run_prefill(w, x, "f64")
+    sl = run_prefill(w, x, "f64", vote_rows=R)
+    np.testing.assert_array_equal(blk["tile_state"], sl["tile_state"])
+    assert (blk["skipped"], blk["visited"]) == (sl["skipped"], sl["visited"])
+    n_sl = w.Br // R
+    mask = sl["slice_mask"]
+    bits = np.unpackbits(mask[..., None], axis=-1)[..., -n_sl:].sum()
+    # Counters: slices holding a valid row. Bits of empty (padding) slices are set
+    # but not counted.
+    n_q = -(-w.L // w.Br)
+    rows_last = w.L - (n_q - 1) * w.Br
+    empty_last = n_sl - (-(-rows_last // R))
+    vis_last = int((mask[:, :, -1, :] != 0).sum())
+    assert sl["slices_visited"] == n_sl * sl["visited"] - empty_last * vis_last
+    assert sl["slices_skipped"] == bits - empty_last * vis_last
+    assert sl["slices_skipped"] >= n_sl * sl["skipped"] - empty_last * vis_last
+    # vote_rows = Br: one slice per tile, same counts as the blocks.
+    assert (blk["slices_skipped"], blk["slices_visited"]) == (blk["skipped"], blk["visited"])
+
+
+def test_slice_vote_planted_case():
+    # 32 query rows, Br = 32, R = 16, Bc = 16, non-causal, scale 1/4.
+    # Rows 0-15 (slice 0) have q = 4 e0, rows 16-31 (slice 1) q = 4 e1.
+    # Key tile 0: key 0 = 8 e0 + 8 e1 (logit 8 for every row).
+    # Key tile 1: key 16 = 7.5 e1 and key 17 = 0: slice 0 sees max logit 0
+    #   (gap 8: passes at ln t = -4), slice 1 sees 7.5 (gap 0.5: fails).
+    # The block is kept, slice 0 skips it, slice 1 keeps it.
+    d, L = 16, 32
+    q = np.zeros((1, 1, L, d), np.float32)
+    q[0, 0, :16, 0] = 4.0
+    q[0, 0, 16:, 1] = 4.0
+    k = np.zeros((1, 1, L, d), np.float32)
+    k[0, 0, 0, 0] = 8.0
+    k[0, 0, 0, 1] = 8.0
+    k[0, 0, 16, 1] = 7.5
+    v = np.ones((1, 1, L, d), np.float32)
+    v[0, 0, 16:, :] = 3.0
+    x = {"q": bf16_bits(q), "k": bf16_bits(k), "v": bf16_bits(v)}
+    tsf = L * math.exp(-4.0)
+    for precision in ("f32", "f64"):
+        got = oracle.prefill(x["q"], x["k"], x["v"], causal=False, sm_scale=0.25, tsf=tsf,
+                             Br=32, Bc=16, vote_rows=16, precision=precision)
+        assert list(got["tile_state"][0, 0, 0]) == [1, 1]
+        assert list(got["slice_mask"][0, 0, 0]) == [0x80, 0x80 | 0b01]
+        assert (got["slices_skipped"], got["slices_visited"]) == (1, 4)
+        # slice 0: only tile 0 -> all V = 1 -> O = 1; lse = ln(e^8 + 15).
+        np.testing.assert_allclose(got["o"][0, 0, :16], 1.0, atol=1e-6)
+        np.testing.assert_allclose(got["lse"][0, 0, :16], math.log(math.exp(8) + 15), atol=1e-5)
+        # slice 1: tile 0 (one key at 8, 15 at 0; V = 1) + tile 1 (one key at
+        # 7.5, 15 at 0; V = 3).
+        num = math.exp(8) + 15 + 3 * (math.exp(7.5) + 15)
+        den = math.exp(8) + 15 + math.exp(7.5) + 15
+        np.testing.assert_allclose(got["o"][0, 0, 16:], num / den, rtol=1e-5)
+        np.testing.assert_allclose(got["lse"][0, 0, 16:], math.log(den), atol=1e-5)
+        blk = oracle.prefill(x["q"], x["k"], x["v"], causal=False, sm_scale=0.25, tsf=tsf,
+                             Br=32, Bc=16, precision=precision)
+        np.testing.assert_allclose(blk["o"][0, 0, :16],
+                                   (math.exp(8) + 15 + 3 * 16) / (math.exp(8) + 15 + 16),
+                                   rtol=1e-5)
+
+
+def test_slice_vote_rejects_bad_rows():
+    w = small_prefill(L=128, Br=64, Bc=64)
+    x = synth.prefill_inputs(w, "lit")
+    for R in (0, 48, 65, 8):   # not a divisor, too large, or more than 7 slices
+        with pytest.raises(ValueError):
+            run_prefill(w, x, vote_rows=R)
