@@ -225,3 +225,54 @@ def slice_restricted_attention(q_bits, k_bits, v_bits, slice_mask, *, causal, sc
     L = S.shape[-1]
     return masked_softmax_attention(S, v_bits,
                                     slice_kept_key_mask(slice_mask, L, Br, Bc, R, causal))
+
+
+def prefill_critical_factors(q_bits, k_bits, *, causal, scale, Br, Bc):
+    """ln of the smallest threshold_scale_factor at which each visited tile is
+    skipped, in closed form (t < 1): the tile is skipped iff every valid row
+    has m_local - prefix_max < ln(tsf / L), i.e. iff
+    ln tsf > max_r (m_local - prefix_max) + ln L. +inf for a tile no factor
+    below L skips (the first tile). Returns [B, H, n_q, n_k] with NaN where
+    the tile is not visited."""
+    S = logits(q_bits, k_bits, scale)
+    B, H, L, _ = S.shape
+    n_q, n_k = -(-L // Br), -(-L // Bc)
+    if causal:
+        S = np.where(causal_mask(L), S, -np.inf)
+    out = np.full((B, H, n_q, n_k), np.nan)
+    for i in range(n_q):
+        r0, r1 = i * Br, min(L, (i + 1) * Br)
+        j_max = min(n_k - 1, ((i + 1) * Br - 1) // Bc) if causal else n_k - 1
+        prefix = np.full((B, H, r1 - r0), -np.inf)
+        for j in range(j_max + 1):
+            ml = S[:, :, r0:r1, j * Bc:min(L, (j + 1) * Bc)].max(axis=-1)
+            with np.errstate(invalid="ignore"):
+                gap = np.where(ml == -np.inf, -np.inf,
+                               np.where(prefix == -np.inf, np.inf, ml - prefix))
+            out[:, :, i, j] = gap.max(axis=-1) + math.log(L)
+            prefix = np.maximum(prefix, ml)
+    return out
+
+
+def decode_critical_factors(q_bits, kc_bits, seqlens, *, scale, Bc, num_splits):
+    """Decode version: joint vote of the G heads, per-split running maximum,
+    t_b = tsf / L_b. [B, Hkv, ceil(Lmax/Bc)], NaN beyond each sequence."""
+    B, Hq, d = q_bits.shape
+    Hkv, Lmax = kc_bits.shape[1], kc_bits.shape[2]
+    G = Hq // Hkv
+    out = np.full((B, Hkv, -(-Lmax // Bc)), np.nan)
+    for b in range(B):
+        Lb = int(seqlens[b])
+        n_k = -(-Lb // Bc)
+        c = -(-n_k // num_splits)
+        for h in range(Hkv):
+            S = decode_logits(q_bits[b, h * G:(h + 1) * G], kc_bits[b, h], Lb, scale)
+            m_loc = np.stack([S[:, j * Bc:min(Lb, (j + 1) * Bc)].max(axis=1) for j in range(n_k)], 1)
+            for s in range(num_splits):
+                prefix = np.full(G, -np.inf)
+                for j in range(s * c, min((s + 1) * c, n_k)):
+                    ml = m_loc[:, j]
+                    gap = np.where(prefix == -np.inf, np.inf, ml - prefix)
+                    out[b, h, j] = gap.max() + math.log(Lb)
+                    prefix = np.maximum(prefix, ml)
+    return out
