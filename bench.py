@@ -275,6 +275,7 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
     readings = [r for r in args.readings.split(",") if r]
     if args.reading not in readings:
         readings.insert(0, args.reading)
+    warp_readings = [r for r in args.warp_vote_readings.split(",") if r]
     dw = decode_workload(args)
 
     # ---- legs of the step: prefill and decode, one per generator reading.
@@ -295,6 +296,21 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
                                       stream=stream)
             legs.append({"name": f"prefill_{rd}", "kind": "prefill", "reading": rd, "t": t,
                          "host": x, "run": run, "launches": 1})
+            if rd in warp_readings:
+                # Same inputs, vote taken per 32-row warp slice.
+                tw = dict(t, o=torch.empty_like(t["q"]),
+                          lse=torch.empty_like(t["lse"]),
+                          cnt=torch.zeros(4, dtype=torch.int64, device=dev))
+
+                def run_w(t=tw, tsf=None, tiles=None):
+                    sk.sskip_attn_prefill_vote(
+                        t["q"], t["k"], t["v"], t["o"], t["lse"], causal=w.causal,
+                        sm_scale=w.scale, threshold_scale_factor=w.tsf if tsf is None else tsf,
+                        Br=w.Br, Bc=w.Bc, vote_rows=32, counts=t["cnt"], tile_state=tiles,
+                        stream=stream)
+                legs.append({"name": f"prefill_{rd}_warp32", "kind": "prefill", "reading": rd,
+                             "vote": "warp32", "t": tw, "host": x, "run": run_w, "launches": 1,
+                             "extra": True})
     if args.only != "prefill":
         for rd in (readings if args.decode_readings == "all" else [args.reading]):
             dx = synth.decode_inputs(dw, rd)
@@ -326,6 +342,8 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
             leg["run"](tiles=tiles)
             c = t["cnt"].cpu().tolist()
             leg["stats"] = {"skipped": c[0], "visited": c[1], **prefill_flops(w, c[1], c[0])}
+            if len(c) == 4:
+                leg["stats"].update(slices_skipped=c[2], slices_visited=c[3])
         else:
             tiles = torch.empty((dw.B, dw.Hkv, -(-dw.Lmax // dw.Bc)), dtype=torch.uint8, device=dev)
             leg["run"](tiles=tiles)
@@ -339,8 +357,10 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
         return {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for n in names}
 
-    def timed(body, steps):
-        """Run `body(events)` steps times after warm-up; device ms per leg, max over ranks."""
+    def timed(body, steps, only=None):
+        """Run `body(events)` steps times after warm-up; device ms per leg
+        (the legs in `only`, default all), max over ranks."""
+        sel = names if only is None else [n for n in names if n in only]
         for _ in range(args.warmup):
             body(new_events())
         barrier()
@@ -348,11 +368,13 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
         for i in range(steps):
             body(evs[i])
         barrier()
-        ms = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in evs) / steps for n in names}
-        return dict(zip(names, reduce_max([ms[n] for n in names], world, dev)))
+        ms = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in evs) / steps for n in sel}
+        return dict(zip(sel, reduce_max([ms[n] for n in sel], world, dev)))
 
     def step(ev, tsf=None):
         for leg in legs:
+            if tsf is not None and leg.get("extra"):
+                continue  # the control at tsf = 0 is the same for both votes
             flush.zero_()
             ev[leg["name"]][0].record(stream)
             leg["run"](tsf=tsf)
@@ -370,7 +392,8 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
     assert sk.sskip_get_status() == sk.SSKIP_OK
 
     # ---- skip-disabled control: the same kernels and inputs at tsf = 0
-    ms_dense = timed(lambda ev: step(ev, tsf=0.0), max(3, args.steps // 3)) \
+    core = [leg["name"] for leg in legs if not leg.get("extra")]
+    ms_dense = timed(lambda ev: step(ev, tsf=0.0), max(3, args.steps // 3), only=core) \
         if not args.no_control else {}
 
     # ---- end to end through the public API: pinned host in, host out
@@ -389,6 +412,7 @@ def time_e2e(legs, flush, stream, new_events, timed, steps):
     """Same steps with each leg's inputs copied host->device from pinned memory
     and its outputs copied back inside the timed region."""
     import torch
+    legs = [leg for leg in legs if not leg.get("extra")]
     h2d = d2h = 0
     for leg in legs:
         t = leg["t"]
@@ -418,7 +442,7 @@ def time_e2e(legs, flush, stream, new_events, timed, steps):
             leg["pin_out"][1].copy_(t["lse"], non_blocking=True)
             ev[leg["name"]][1].record(stream)
 
-    return timed(e2e_step, steps), (h2d, d2h)
+    return timed(e2e_step, steps, only=[leg["name"] for leg in legs]), (h2d, d2h)
 
 
 def report(args, w, dw, world, legs, ms, ms_dense, ems, io_bytes, peaks, peak_kind,
@@ -452,7 +476,15 @@ def report(args, w, dw, world, legs, ms, ms_dense, ems, io_bytes, peaks, peak_ki
                      ideal_speedup=ideal)
         if n in ems:
             b["e2e_ms"] = ems[n]
-        (pre if leg["kind"] == "prefill" else dec)[leg["reading"]] = b
+        key = leg["reading"]
+        if leg.get("vote"):
+            key = f"{key}_{leg['vote']}"
+            b.update(vote_rows=32, slice_skip_fraction=s["slices_skipped"] / max(1, s["slices_visited"]),
+                     slices_skipped=s["slices_skipped"], slices_visited=s["slices_visited"])
+            blk = f"prefill_{leg['reading']}"
+            if blk in ms:
+                b["speedup_vs_block_vote"] = ms[blk] / ms[n]
+        (pre if leg["kind"] == "prefill" else dec)[key] = b
     head = args.reading
     if pre:
         hs = next(leg["stats"] for leg in legs if leg["name"] == f"prefill_{head}")
@@ -578,6 +610,8 @@ def main(argv=None):
     ap.add_argument("--no-control", action="store_true",
                     help="skip the tsf = 0 (skipping disabled) control timing")
     ap.add_argument("--decode-readings", choices=["all", "headline"], default="all")
+    ap.add_argument("--warp-vote-readings", default="lit,rms",
+                    help="readings also timed with the per-warp (32-row) vote; '' for none")
     ap.add_argument("--sweep", action="store_true",
                     help="threshold sweep of --prefill (default: the 128K long prefill)")
     args = ap.parse_args(argv)

@@ -24,7 +24,8 @@ LIB_PATH = os.path.join(_PKG, "libsskip_attn.so")
 SSKIP_OK, SSKIP_ERR_INVALID_ARG, SSKIP_ERR_UNSUPPORTED, SSKIP_ERR_CUDA, SSKIP_ERR_TIMEOUT = range(5)
 
 EXPORTS = ("sskip_version", "sskip_status_string", "sskip_device_supported",
-           "sskip_attn_prefill", "sskip_attn_prefill_ex", "sskip_attn_decode_workspace_size",
+           "sskip_attn_prefill", "sskip_attn_prefill_ex", "sskip_attn_prefill_vote",
+           "sskip_attn_decode_workspace_size",
            "sskip_attn_decode", "sskip_attn_decode_ex", "sskip_attn_decode_noalloc",
            "sskip_get_status", "sskip_selftest_watchdog")
 
@@ -60,7 +61,9 @@ def lib() -> ctypes.CDLL:
         L.sskip_attn_prefill.restype = I
         L.sskip_attn_prefill.argtypes = pre + [P]
         L.sskip_attn_prefill_ex.restype = I
-        L.sskip_attn_prefill_ex.argtypes = pre + [P, P]
+        L.sskip_attn_prefill_ex.argtypes = pre[:-1] + [P, P, P]
+        L.sskip_attn_prefill_vote.restype = I
+        L.sskip_attn_prefill_vote.argtypes = pre[:-1] + [I, P, P, P, P]
         L.sskip_attn_decode_workspace_size.restype = Z
         L.sskip_attn_decode_workspace_size.argtypes = [I, I, I, I]
         dec = [P, P, P, P, P, P, I, I, I, I, I, F, F, I, I, P, Z, P]
@@ -123,6 +126,24 @@ def sskip_attn_prefill(q, k, v, o, lse, *, causal: bool, sm_scale: float,
     _check(rc, "sskip_attn_prefill")
 
 
+def sskip_attn_prefill_vote(q, k, v, o, lse, *, causal: bool, sm_scale: float,
+                            threshold_scale_factor: float, Br: int = 128, Bc: int = 128,
+                            vote_rows: int = 32, counts=None, tile_state=None, slice_mask=None,
+                            stream=None) -> None:
+    """Marshal the prefill tensors plus vote_rows, counts int64[4] (optional),
+    tile_state and slice_mask uint8 (optional) into sskip_attn_prefill_vote."""
+    for t in (q, k, v, o):
+        _bf16_view(t)
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    rc = lib().sskip_attn_prefill_vote(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq,
+                                       Hkv, L, d, int(bool(causal)), float(sm_scale),
+                                       float(threshold_scale_factor), int(Br), int(Bc),
+                                       int(vote_rows), _ptr(counts), _ptr(tile_state),
+                                       _ptr(slice_mask), _stream(stream))
+    _check(rc, "sskip_attn_prefill_vote")
+
+
 def sskip_attn_decode_workspace_size(B: int, Hq: int, d: int, num_splits: int) -> int:
     return int(lib().sskip_attn_decode_workspace_size(B, Hq, d, num_splits))
 
@@ -173,19 +194,31 @@ def sskip_selftest_watchdog(limit_us: int, stream=None) -> None:
 
 # -------------------------------------------------------------- conveniences
 def prefill(q, k, v, *, causal: bool, sm_scale: float, threshold_scale_factor: float,
-            Br: int = 128, Bc: int = 128, with_tiles: bool = False, stream=None) -> dict:
-    """Allocate outputs with torch and run sskip_attn_prefill on q's device."""
+            Br: int = 128, Bc: int = 128, with_tiles: bool = False, vote_rows: int | None = None,
+            stream=None) -> dict:
+    """Allocate outputs with torch and run sskip_attn_prefill on q's device;
+    with ``vote_rows`` (Br or 32), run sskip_attn_prefill_vote instead and
+    also return the four counters and the slice record."""
     B, Hq, L, d = q.shape
     o = torch.empty((B, Hq, L, d), dtype=q.dtype, device=q.device)
     lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
-    counts = torch.zeros(2, dtype=torch.int64, device=q.device)
     tiles = None
+    rec_shape = (B, Hq, -(-L // Br), -(-L // Bc))
     if with_tiles:
-        tiles = torch.empty((B, Hq, -(-L // Br), -(-L // Bc)), dtype=torch.uint8, device=q.device)
-    sskip_attn_prefill(q, k, v, o, lse, causal=causal, sm_scale=sm_scale,
-                       threshold_scale_factor=threshold_scale_factor, Br=Br, Bc=Bc,
-                       skip_count=counts, tile_state=tiles, stream=stream)
-    return {"o": o, "lse": lse, "counts": counts, "tile_state": tiles}
+        tiles = torch.empty(rec_shape, dtype=torch.uint8, device=q.device)
+    if vote_rows is None:
+        counts = torch.zeros(2, dtype=torch.int64, device=q.device)
+        sskip_attn_prefill(q, k, v, o, lse, causal=causal, sm_scale=sm_scale,
+                           threshold_scale_factor=threshold_scale_factor, Br=Br, Bc=Bc,
+                           skip_count=counts, tile_state=tiles, stream=stream)
+        return {"o": o, "lse": lse, "counts": counts, "tile_state": tiles}
+    counts = torch.zeros(4, dtype=torch.int64, device=q.device)
+    smask = torch.empty(rec_shape, dtype=torch.uint8, device=q.device) if with_tiles else None
+    sskip_attn_prefill_vote(q, k, v, o, lse, causal=causal, sm_scale=sm_scale,
+                            threshold_scale_factor=threshold_scale_factor, Br=Br, Bc=Bc,
+                            vote_rows=vote_rows, counts=counts, tile_state=tiles,
+                            slice_mask=smask, stream=stream)
+    return {"o": o, "lse": lse, "counts": counts, "tile_state": tiles, "slice_mask": smask}
 
 
 def decode(q, kcache, vcache, seqlens, *, sm_scale: float, threshold_scale_factor: float,

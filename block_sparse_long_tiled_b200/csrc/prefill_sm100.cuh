@@ -46,8 +46,11 @@ namespace sskip {
 struct PrefillParams {
   __nv_bfloat16* o;            // [B, Hq, L, D]
   float* lse;                  // [B, Hq, L]
-  unsigned long long* counts;  // {skipped, visited} or null
+  unsigned long long* counts;  // {skipped, visited[, slices skipped, slices visited]} or null
   uint8_t* tile_state;         // [B, Hq, n_q, n_k] or null
+  uint8_t* slice_mask;         // [B, Hq, n_q, n_k] or null: 0x80 | slices that skipped
+  int slice_vote;              // 1: each 32-row warp slice votes alone
+  int n_counts;                // 2 or 4 entries in counts
   int B, Hq, Hkv, L, G;
   int n_q;                     // ceil(L / Br)
   int n_k;                     // ceil(L / Bc)
@@ -392,7 +395,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const float scale = p.scale_log2;
 
     float m_run = -INFINITY, m_ref = -INFINITY, l_run = 0.f;
-    long long n_vis = 0, n_skip = 0;
+    long long n_vis = 0, n_skip = 0, n_svis = 0, n_sskip = 0;
 
     auto post_vote = [&](int j, bool kept) {  // elected thread only
       const int vslot = j % VS;
@@ -446,22 +449,35 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
       for (int g = 0; g < NGRP; ++g) {
         bool all = true;
+        uint32_t bits = 0;
 #pragma unroll
-        for (int w = 0; w < WPG; ++w) all = all && (wflag[(wg * 2 + (j & 1)) * 4 + g * WPG + w] != 0);
+        for (int w = 0; w < WPG; ++w) {
+          const bool f = wflag[(wg * 2 + (j & 1)) * 4 + g * WPG + w] != 0;
+          all = all && f;
+          bits |= f ? (1u << w) : 0u;
+        }
         const bool vis = j <= g_jmax[g];
         g_kept[g] = vis && !all;
         tile_kept = tile_kept || g_kept[g];
         if (elected && vis) {
           ++n_vis;
           n_skip += all ? 1 : 0;
-          if (p.tile_state)
-            p.tile_state[(((size_t)b * p.Hq + hq) * p.n_q + g_tile[g]) * p.n_k + j] = all ? 2 : 1;
+          const size_t rec = (((size_t)b * p.Hq + hq) * p.n_q + g_tile[g]) * p.n_k + j;
+          if (p.tile_state) p.tile_state[rec] = all ? 2 : 1;
+          if (p.slice_mask) p.slice_mask[rec] = uint8_t(0x80u | (p.slice_vote ? bits : (all ? 1u : 0u)));
         }
+      }
+      // Slice counters: warps holding at least one valid row of a visiting group.
+      if (lane == 0 && gvis && row0 + 128 * wg + wq * 32 < p.L) {
+        ++n_svis;
+        n_sskip += wall ? 1 : 0;
       }
       if (elected) post_vote(j, tile_kept);
 
       if (tile_kept) {
-        const bool mine = g_kept[grp] && row_in;
+        // Block vote: every row of a kept group updates.  Warp vote: only the
+        // rows of a warp slice that did not pass.
+        const bool mine = row_in && (p.slice_vote ? (gvis && !wall) : g_kept[grp]);
         float alpha = 1.f;
         bool rescale = false;
         if (mine) {
@@ -492,64 +508,74 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             tmem_st32(tO + c * 32, w32);
           }
         }
-        uint64_t sum2v[SSKIP_PF_NACC];
+        if (__all_sync(0xffffffffu, !mine)) {
+          // No row of this warp takes part (its slice or group skipped the
+          // tile, or it is padding): P = 0 without any exponential.
+          uint32_t z[32];
 #pragma unroll
-        for (int a = 0; a < SSKIP_PF_NACC; ++a) sum2v[a] = f2pack(0.f, 0.f);
-        float suma = 0.f, sumb = 0.f;
+          for (int i = 0; i < 32; ++i) z[i] = 0u;
 #pragma unroll
-        for (int h = 0; h < BC / 64; ++h) {  // 64 keys -> 32 packed columns at a time
-          uint32_t pk[32];
-          float* sh = s;
-          uint32_t rr[64];
-          if constexpr (SSKIP_PF_RELOAD) {
-            // The row max is known; re-read this half of S (its columns are
-            // still intact: P of half h lands in columns [32h, 32h + 32)).
-            tmem_ld32_async(tS + h * 64, rr);
-            tmem_ld32_async(tS + h * 64 + 32, rr + 32);
-            tmem_wait_ld_tie64(rr);
-            sh = reinterpret_cast<float*>(rr) - h * 64;
-            if (need_mask) {
+          for (int h = 0; h < BC / 64; ++h) tmem_st32(tS + h * 32, z);
+        } else {
+          uint64_t sum2v[SSKIP_PF_NACC];
 #pragma unroll
-              for (int c = 0; c < 64; ++c) {
-                const int key = key0 + h * 64 + c;
-                if (key >= p.L || (CAUSAL && key > row)) rr[c] = __float_as_uint(-INFINITY);
+          for (int a = 0; a < SSKIP_PF_NACC; ++a) sum2v[a] = f2pack(0.f, 0.f);
+          float suma = 0.f, sumb = 0.f;
+#pragma unroll
+          for (int h = 0; h < BC / 64; ++h) {  // 64 keys -> 32 packed columns at a time
+            uint32_t pk[32];
+            float* sh = s;
+            uint32_t rr[64];
+            if constexpr (SSKIP_PF_RELOAD) {
+              // The row max is known; re-read this half of S (its columns are
+              // still intact: P of half h lands in columns [32h, 32h + 32)).
+              tmem_ld32_async(tS + h * 64, rr);
+              tmem_ld32_async(tS + h * 64 + 32, rr + 32);
+              tmem_wait_ld_tie64(rr);
+              sh = reinterpret_cast<float*>(rr) - h * 64;
+              if (need_mask) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                  const int key = key0 + h * 64 + c;
+                  if (key >= p.L || (CAUSAL && key > row)) rr[c] = __float_as_uint(-INFINITY);
+                }
               }
             }
-          }
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int c = h * 32 + i;
-            float p0, p1;
-            if (SSKIP_PF_SCALAR && !exp2_on_fma(c)) {
-              p0 = ex2_approx(fmaf(sh[2 * c], scale, nref));
-              p1 = ex2_approx(fmaf(sh[2 * c + 1], scale, nref));
-              suma += p0;
-              sumb += p1;
-            } else {
-              const uint64_t x2 = ffma2(f2pack(sh[2 * c], sh[2 * c + 1]), scale2, nref2);
-              if (exp2_on_fma(c)) {
-                f2unpack(exp2_fma2(x2), p0, p1);
+            for (int i = 0; i < 32; ++i) {
+              const int c = h * 32 + i;
+              float p0, p1;
+              if (SSKIP_PF_SCALAR && !exp2_on_fma(c)) {
+                p0 = ex2_approx(fmaf(sh[2 * c], scale, nref));
+                p1 = ex2_approx(fmaf(sh[2 * c + 1], scale, nref));
+                suma += p0;
+                sumb += p1;
               } else {
-                float x0, x1;
-                f2unpack(x2, x0, x1);
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
+                const uint64_t x2 = ffma2(f2pack(sh[2 * c], sh[2 * c + 1]), scale2, nref2);
+                if (exp2_on_fma(c)) {
+                  f2unpack(exp2_fma2(x2), p0, p1);
+                } else {
+                  float x0, x1;
+                  f2unpack(x2, x0, x1);
+                  p0 = ex2_approx(x0);
+                  p1 = ex2_approx(x1);
+                }
+                sum2v[c % SSKIP_PF_NACC] = fadd2(sum2v[c % SSKIP_PF_NACC], f2pack(p0, p1));
               }
-              sum2v[c % SSKIP_PF_NACC] = fadd2(sum2v[c % SSKIP_PF_NACC], f2pack(p0, p1));
+              if (SSKIP_PF_PACK_PRMT)
+                pk[i] = pack_bf16x2_halfup(p0, p1);
+              else
+                pk[i] = pack_bf16x2(p0, p1);
             }
-            if (SSKIP_PF_PACK_PRMT)
-              pk[i] = pack_bf16x2_halfup(p0, p1);
-            else
-              pk[i] = pack_bf16x2(p0, p1);
+            tmem_st32(tS + h * 32, pk);
           }
-          tmem_st32(tS + h * 32, pk);
-        }
-        uint64_t sum2 = sum2v[0];
+          uint64_t sum2 = sum2v[0];
 #pragma unroll
-        for (int a = 1; a < SSKIP_PF_NACC; ++a) sum2 = fadd2(sum2, sum2v[a]);
-        float sa, sb;
-        f2unpack(sum2, sa, sb);
-        l_run += mine ? ((sa + sb) + (suma + sumb)) : 0.f;
+          for (int a = 1; a < SSKIP_PF_NACC; ++a) sum2 = fadd2(sum2, sum2v[a]);
+          float sa, sb;
+          f2unpack(sum2, sa, sb);
+          l_run += mine ? ((sa + sb) + (suma + sumb)) : 0.f;
+        }
         tmem_st_wait();
         tc_fence_before();
         named_bar_sync(bar_id, 128);
@@ -590,6 +616,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (elected && p.counts) {
       atomicAdd(&p.counts[0], (unsigned long long)n_skip);
       atomicAdd(&p.counts[1], (unsigned long long)n_vis);
+      if (p.n_counts == 4 && !p.slice_vote) {  // one slice per block
+        atomicAdd(&p.counts[2], (unsigned long long)n_skip);
+        atomicAdd(&p.counts[3], (unsigned long long)n_vis);
+      }
+    }
+    if (lane == 0 && p.counts && p.n_counts == 4 && p.slice_vote && n_svis > 0) {
+      atomicAdd(&p.counts[2], (unsigned long long)n_sskip);
+      atomicAdd(&p.counts[3], (unsigned long long)n_svis);
     }
   }
 

@@ -139,14 +139,16 @@ SSKIP_API int sskip_device_supported(int device) {
   return (prop.major == 10 && prop.minor == 0) ? SSKIP_OK : SSKIP_ERR_UNSUPPORTED;
 }
 
-SSKIP_API int sskip_attn_prefill_ex(const void* q, const void* k, const void* v, void* o,
-                                    float* lse, int B, int Hq, int Hkv, int L, int d, int causal,
-                                    float sm_scale, float threshold_scale_factor, int Br, int Bc,
-                                    unsigned long long* skip_count, uint8_t* tile_state,
-                                    void* stream) {
+namespace sskip {
+namespace {
+
+int prefill_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                 int Hkv, int L, int d, int causal, float sm_scale, float threshold_scale_factor,
+                 int Br, int Bc, int vote_rows, unsigned long long* counts, int n_counts,
+                 uint8_t* tile_state, uint8_t* slice_mask, void* stream) {
   if (!q || !k || !v || !o || !lse) return SSKIP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(skip_count) & 7u))
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(counts) & 7u))
     return SSKIP_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0) return SSKIP_ERR_INVALID_ARG;
   if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SSKIP_ERR_INVALID_ARG;
@@ -154,6 +156,7 @@ SSKIP_API int sskip_attn_prefill_ex(const void* q, const void* k, const void* v,
     return SSKIP_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return SSKIP_ERR_UNSUPPORTED;
   if (!((Br == 64 && Bc == 64) || (Br == 128 && Bc == 128))) return SSKIP_ERR_UNSUPPORTED;
+  if (vote_rows != Br && vote_rows != 32) return SSKIP_ERR_UNSUPPORTED;
   const long long n_units = (L + kPfUnitRows - 1) / kPfUnitRows;
   if ((long long)B * Hq * n_units >= (1ll << 31) || (long long)B * Hq >= (1ll << 31))
     return SSKIP_ERR_UNSUPPORTED;
@@ -168,8 +171,11 @@ SSKIP_API int sskip_attn_prefill_ex(const void* q, const void* k, const void* v,
   PrefillParams p{};
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
-  p.counts = skip_count;
+  p.counts = counts;
+  p.n_counts = n_counts;
   p.tile_state = tile_state;
+  p.slice_mask = slice_mask;
+  p.slice_vote = vote_rows != Br;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.G = Hq / Hkv;
   p.n_q = (L + Br - 1) / Br;
   p.n_k = (L + Bc - 1) / Bc;
@@ -179,10 +185,14 @@ SSKIP_API int sskip_attn_prefill_ex(const void* q, const void* k, const void* v,
   p.log2_t = p.t_positive ? (float)std::log2((double)threshold_scale_factor / (double)L)
                           : -INFINITY;
 
-  if (skip_count && cudaMemsetAsync(skip_count, 0, 2 * sizeof(unsigned long long), st) != cudaSuccess)
+  if (counts &&
+      cudaMemsetAsync(counts, 0, (size_t)n_counts * sizeof(unsigned long long), st) != cudaSuccess)
     return SSKIP_ERR_CUDA;
   if (tile_state &&
       cudaMemsetAsync(tile_state, 0, (size_t)B * Hq * p.n_q * p.n_k, st) != cudaSuccess)
+    return SSKIP_ERR_CUDA;
+  if (slice_mask &&
+      cudaMemsetAsync(slice_mask, 0, (size_t)B * Hq * p.n_q * p.n_k, st) != cudaSuccess)
     return SSKIP_ERR_CUDA;
 
   const bool c = causal != 0;
@@ -194,6 +204,27 @@ SSKIP_API int sskip_attn_prefill_ex(const void* q, const void* k, const void* v,
                                      : launch_prefill<128, 64, 64, false>(mq, mk, mv, p, st);
   return c ? launch_prefill<64, 64, 64, true>(mq, mk, mv, p, st)
            : launch_prefill<64, 64, 64, false>(mq, mk, mv, p, st);
+}
+
+}  // namespace
+}  // namespace sskip
+
+SSKIP_API int sskip_attn_prefill_ex(const void* q, const void* k, const void* v, void* o,
+                                    float* lse, int B, int Hq, int Hkv, int L, int d, int causal,
+                                    float sm_scale, float threshold_scale_factor, int Br, int Bc,
+                                    unsigned long long* skip_count, uint8_t* tile_state,
+                                    void* stream) {
+  return prefill_impl(q, k, v, o, lse, B, Hq, Hkv, L, d, causal, sm_scale, threshold_scale_factor,
+                      Br, Bc, Br, skip_count, 2, tile_state, nullptr, stream);
+}
+
+SSKIP_API int sskip_attn_prefill_vote(const void* q, const void* k, const void* v, void* o,
+                                      float* lse, int B, int Hq, int Hkv, int L, int d, int causal,
+                                      float sm_scale, float threshold_scale_factor, int Br, int Bc,
+                                      int vote_rows, unsigned long long* counts,
+                                      uint8_t* tile_state, uint8_t* slice_mask, void* stream) {
+  return prefill_impl(q, k, v, o, lse, B, Hq, Hkv, L, d, causal, sm_scale, threshold_scale_factor,
+                      Br, Bc, vote_rows, counts, 4, tile_state, slice_mask, stream);
 }
 
 SSKIP_API int sskip_attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,

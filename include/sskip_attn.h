@@ -100,6 +100,34 @@ int sskip_attn_prefill_ex(const void* q, const void* k, const void* v, void* o, 
                           unsigned long long* skip_count, uint8_t* tile_state, void* stream);
 
 /*
+ * Prefill with a choice of vote granularity.  vote_rows = Br is the block
+ * vote of sskip_attn_prefill.  vote_rows = 32 takes the same test per warp
+ * slice of 32 query rows, the granularity of the "稀疏 Warp 在线 Softmax"
+ * stage in the SpargeAttn article (its local-vs-global maximum test, taken
+ * per warp): each slice of a tile passes or fails on its own rows, and a
+ * slice that passes leaves its rows' m, l and O untouched (no exponentials
+ * for it).  The tile's V load and its P.V still run unless every slice of
+ * the tile passes, so the block decisions (and the tile_state record) equal
+ * those of the block vote whenever t < 1; the outputs differ only in the
+ * small terms the passing slices drop.
+ *
+ *   vote_rows: Br or 32; anything else is SSKIP_ERR_UNSUPPORTED.
+ *   counts: optional device uint64[4] = {skipped tiles, visited tiles,
+ *     skipped slices, visited slices}; a slice is counted when it holds at
+ *     least one row < L.  With vote_rows = Br the slices are the tiles.
+ *   tile_state: optional, as in sskip_attn_prefill_ex.
+ *   slice_mask: optional device uint8 [B, Hq, ceil(L/Br), ceil(L/Bc)]:
+ *     0 = tile not visited, else 0x80 | bit s set when slice s (rows
+ *     [s * vote_rows, (s + 1) * vote_rows) of the query tile) skipped it.  A
+ *     slice with no row < L passes vacuously (its bit is set).
+ */
+int sskip_attn_prefill_vote(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int Hq, int Hkv, int L, int d, int causal, float sm_scale,
+                            float threshold_scale_factor, int Br, int Bc, int vote_rows,
+                            unsigned long long* counts, uint8_t* tile_state,
+                            uint8_t* slice_mask, void* stream);
+
+/*
  * Decode: one new query token per sequence against a contiguous KV cache,
  * split over the key axis and merged by log-sum-exp (the bandwidth-bound
  * phase of the article's "Skip Softmax 带来了哪些实战好处" section: a skipped

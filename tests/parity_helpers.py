@@ -78,3 +78,59 @@ def unit_restricted_reference(x, w, b, hq, i, kept_tiles):
     P = np.where(allowed, np.exp(S - m), 0.0)
     l = P.sum(axis=1, keepdims=True)
     return (P @ v) / l, (m + np.log(l))[:, 0]
+
+
+def unit_slice_restricted_reference(x, w, b, hq, i, slice_mask_row, R):
+    """fp64 attention of query tile i of (b, hq) where row r sees key tile j
+    iff the tile was visited (bit 7 of slice_mask_row[j]) and r's R-row slice
+    did not skip it (bit (r - i*Br) // R clear)."""
+    G = w.Hq // w.Hkv
+    r0, r1 = i * w.Br, min(w.L, (i + 1) * w.Br)
+    q = synth.bf16_to_f32(x["q"][b, hq, r0:r1]).astype(np.float64)
+    k = synth.bf16_to_f32(x["k"][b, hq // G]).astype(np.float64)
+    v = synth.bf16_to_f32(x["v"][b, hq // G]).astype(np.float64)
+    S = w.scale * q @ k.T
+    keys = np.arange(w.L)
+    sm = np.asarray(slice_mask_row).astype(np.int64)
+    bit = (np.arange(r1 - r0) // R)[:, None]
+    tile_of_key = keys // w.Bc
+    visited = (sm[tile_of_key] & 0x80) != 0
+    skipped = ((sm[tile_of_key][None, :] >> bit) & 1) != 0
+    allowed = visited[None, :] & ~skipped
+    if w.causal:
+        allowed &= keys[None, :] <= np.arange(r0, r1)[:, None]
+    S = np.where(allowed, S, -np.inf)
+    m = S.max(axis=1, keepdims=True)
+    P = np.where(allowed, np.exp(S - m), 0.0)
+    l = P.sum(axis=1, keepdims=True)
+    return (P @ v) / l, (m + np.log(l))[:, 0]
+
+
+def unit_slice_margins(x, w, b, hq, i, R, tsf):
+    """fp64 margin min_r (ln t - (m_local - m_run)) of every R-row slice of
+    query tile i on every key tile, with m_run the prefix maximum (the closed
+    form of the running maximum while t < 1). [n_slices, n_k]; +inf where the
+    slice has no valid row or the tile is not visited."""
+    G = w.Hq // w.Hkv
+    r0, r1 = i * w.Br, min(w.L, (i + 1) * w.Br)
+    q = synth.bf16_to_f32(x["q"][b, hq, r0:r1]).astype(np.float64)
+    k = synth.bf16_to_f32(x["k"][b, hq // G]).astype(np.float64)
+    S = w.scale * q @ k.T
+    if w.causal:
+        S = np.where(np.arange(w.L)[None, :] <= np.arange(r0, r1)[:, None], S, -np.inf)
+    ln_t = math.log(tsf / w.L) if tsf > 0 else -math.inf
+    n_k = -(-w.L // w.Bc)
+    j_max = min(n_k - 1, ((i + 1) * w.Br - 1) // w.Bc) if w.causal else n_k - 1
+    n_sl = w.Br // R
+    out = np.full((n_sl, n_k), np.inf)
+    prefix = np.full(r1 - r0, -np.inf)
+    for j in range(j_max + 1):
+        ml = S[:, j * w.Bc:min(w.L, (j + 1) * w.Bc)].max(axis=1)
+        with np.errstate(invalid="ignore"):
+            mg = np.where(prefix == -np.inf, -np.inf, ln_t - (ml - prefix))
+        for s in range(n_sl):
+            a, e = s * R, min(r1 - r0, (s + 1) * R)
+            if a < e:
+                out[s, j] = mg[a:e].min()
+        prefix = np.maximum(prefix, ml)
+    return out
