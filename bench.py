@@ -580,6 +580,199 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def run_calibration(args):
+    """Calibrate the factor to target skip ratios (one recording pass plus
+    the host selection), then time the kernel at each calibrated factor."""
+    import torch
+    import block_sparse_long_tiled_b200 as sk
+    dev = torch.device("cuda", 0)
+    peaks, _ = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    td = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev).view(
+        torch.bfloat16)
+    targets = [float(t) for t in args.targets.split(",") if t]
+
+    def time_it(fn):
+        ts = []
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ts.append(a.elapsed_time(b))
+        return float(np.median(ts))
+
+    w = synth.PREFILL_WORKLOADS[args.prefill]
+    for rd in [r for r in args.readings.split(",") if r]:
+        x = synth.prefill_inputs(w, rd)
+        q, k, v = td(x["q"]), td(x["k"]), td(x["v"])
+        del x
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
+        cnt = torch.zeros(2, dtype=torch.int64, device=dev)
+
+        def run(f):
+            sk.sskip_attn_prefill(q, k, v, o, lse, causal=w.causal, sm_scale=w.scale,
+                                  threshold_scale_factor=f, Br=w.Br, Bc=w.Bc, skip_count=cnt)
+        dense_ms = time_it(lambda: run(0.0))
+        for tgt in targets:
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            try:
+                r = sk.calibrate_prefill(q, k, v, causal=w.causal, sm_scale=w.scale,
+                                         target_ratio=tgt, Br=w.Br, Bc=w.Bc)
+            except sk.SSkipError as e:
+                print(json.dumps({"calibration": w.name, "reading": rd, "target": tgt,
+                                  "unreachable": str(e)}), flush=True)
+                continue
+            cal_s = time.perf_counter() - t0
+            ms = time_it(lambda: run(r["factor"]))
+            c = cnt.cpu().tolist()
+            f = prefill_flops(w, c[1], c[0])
+            s = c[0] / max(1, c[1])
+            print(json.dumps({"calibration": w.name, "reading": rd, "target": tgt,
+                              "threshold_scale_factor": r["factor"],
+                              "predicted_ratio": r["achieved_ratio"], "skip_fraction": s,
+                              "calibration_wall_s": cal_s, "ms": ms, "ms_dense": dense_ms,
+                              "speedup_vs_dense": dense_ms / ms,
+                              "ideal_speedup": 1.0 / (1.0 - s / 2.0),
+                              "executed_tflops": f["executed"] / ms / 1e9,
+                              "executed_frac_of_peak": f["executed"] / ms / 1e9 / peak}),
+                  flush=True)
+        del q, k, v, o
+        torch.cuda.empty_cache()
+
+    dw = decode_workload(args)
+    for rd in [r for r in args.readings.split(",") if r]:
+        dx = synth.decode_inputs(dw, rd)
+        q, kc, vc = td(dx["q"]), td(dx["kcache"]), td(dx["vcache"])
+        lens = torch.from_numpy(dx["seqlens"]).to(dev)
+        o = torch.empty((dw.B, dw.Hq, dw.d), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((dw.B, dw.Hq), dtype=torch.float32, device=dev)
+        ws = torch.empty(sk.sskip_attn_decode_workspace_size(dw.B, dw.Hq, dw.d, dw.num_splits),
+                         dtype=torch.uint8, device=dev)
+        cnt = torch.zeros(2, dtype=torch.int64, device=dev)
+        tiles = torch.empty((dw.B, dw.Hkv, -(-dw.Lmax // dw.Bc)), dtype=torch.uint8, device=dev)
+
+        def run_d(f, rec=None):
+            sk.sskip_attn_decode(q, kc, vc, lens, o, lse, sm_scale=dw.scale,
+                                 threshold_scale_factor=f, Bc=dw.Bc, num_splits=dw.num_splits,
+                                 workspace=ws, skip_count=cnt, tile_state=rec)
+        dense_ms = time_it(lambda: run_d(0.0))
+        for tgt in targets:
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            try:
+                r = sk.calibrate_decode(q, kc, vc, lens, sm_scale=dw.scale, target_ratio=tgt,
+                                        Bc=dw.Bc, num_splits=dw.num_splits)
+            except sk.SSkipError as e:
+                print(json.dumps({"calibration": dw.name, "reading": rd, "target": tgt,
+                                  "unreachable": str(e)}), flush=True)
+                continue
+            cal_s = time.perf_counter() - t0
+            run_d(r["factor"], tiles)
+            by = decode_bytes(dw, dx["seqlens"], tiles.cpu().numpy())
+            ms = time_it(lambda: run_d(r["factor"]))
+            c = cnt.cpu().tolist()
+            print(json.dumps({"calibration": dw.name, "reading": rd, "target": tgt,
+                              "threshold_scale_factor": r["factor"],
+                              "predicted_ratio": r["achieved_ratio"],
+                              "skip_fraction": c[0] / max(1, c[1]), "calibration_wall_s": cal_s,
+                              "ms": ms, "ms_dense": dense_ms, "speedup_vs_dense": dense_ms / ms,
+                              "ideal_speedup": by["total_dense"] / by["total"],
+                              "gbs_actually_moved": by["total"] / ms / 1e6,
+                              "frac_of_hbm": by["total"] / ms / 1e6 / hbm}), flush=True)
+        del q, kc, vc, dx
+        torch.cuda.empty_cache()
+
+
+def run_reorder(args):
+    """Video prefill in raster and in Hilbert token order (block and per-warp
+    votes): skip fractions, attention time, and the time and bandwidth of the
+    row gathers (Q, K, V) and scatters (O, lse) that reorder the tokens."""
+    import torch
+    import block_sparse_long_tiled_b200 as sk
+    dev = torch.device("cuda", 0)
+    peaks, _ = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    w = synth.VIDEO_DIT_PREFILL if args.prefill == synth.LLAMA8B_PREFILL_16K.name \
+        else synth.PREFILL_WORKLOADS[args.prefill]
+    if args.tsf is not None:
+        w = w.replace(tsf=args.tsf)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    td = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev).view(
+        torch.bfloat16)
+    x = synth.prefill_inputs(w, args.reading)
+    q, k, v = td(x["q"]), td(x["k"]), td(x["v"])
+    del x
+    perm_h = sk.sskip_hilbert3d_order(*w.video_grid, w.L)
+    perm = torch.from_numpy(perm_h).to(dev)
+    qp, kp, vp = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    o, op = torch.empty_like(q), torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
+    lsep = torch.empty_like(lse)
+    cnt = torch.zeros(4, dtype=torch.int64, device=dev)
+
+    def time_it(fn):
+        ts = []
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ts.append(a.elapsed_time(b))
+        return float(np.median(ts))
+
+    def gather():
+        for a, b in ((q, qp), (k, kp), (v, vp)):
+            sk.sskip_permute_rows(a, b, perm, scatter=False)
+
+    def scatter():
+        sk.sskip_permute_rows(op, o, perm, scatter=True)
+        sk.sskip_permute_rows(lsep.unsqueeze(-1), lse.unsqueeze(-1), perm, scatter=True)
+
+    gather()
+    g_ms = time_it(gather)
+    s_ms = time_it(scatter)
+    g_bytes = 3 * 2 * q.numel() * q.element_size()
+    s_bytes = 2 * (o.numel() * o.element_size() + lse.numel() * 4)
+    rows = []
+    for order, (qq, kk, vv, oo, ll) in (("raster", (q, k, v, o, lse)),
+                                        ("hilbert", (qp, kp, vp, op, lsep))):
+        for vote in (w.Br, 32):
+            def run(f=w.tsf):
+                sk.sskip_attn_prefill_vote(qq, kk, vv, oo, ll, causal=w.causal,
+                                           sm_scale=w.scale, threshold_scale_factor=f, Br=w.Br,
+                                           Bc=w.Bc, vote_rows=vote, counts=cnt)
+            run()
+            c = cnt.cpu().tolist()
+            ms = time_it(run)
+            f = prefill_flops(w, c[1], c[0])
+            rows.append({"order": order, "vote_rows": vote, "ms": ms,
+                         "skip_fraction": c[0] / c[1], "slice_skip_fraction": c[2] / c[3],
+                         "executed_tflops": f["executed"] / ms / 1e9,
+                         "executed_frac_of_peak": f["executed"] / ms / 1e9 / peak,
+                         "dense_equiv_tflops": f["dense"] / ms / 1e9})
+    dense_ms = time_it(lambda: sk.sskip_attn_prefill(q, k, v, o, lse, causal=w.causal,
+                                                     sm_scale=w.scale, threshold_scale_factor=0.0,
+                                                     Br=w.Br, Bc=w.Bc))
+    print(json.dumps({"reorder": w.name, "reading": args.reading,
+                      "threshold_scale_factor": w.tsf, "ms_dense": dense_ms,
+                      "gather_qkv_ms": g_ms, "gather_gbs": g_bytes / g_ms / 1e6,
+                      "gather_frac_of_hbm": g_bytes / g_ms / 1e6 / hbm,
+                      "scatter_o_lse_ms": s_ms, "scatter_gbs": s_bytes / s_ms / 1e6,
+                      "runs": rows}), flush=True)
+
+
 def decode_workload(args):
     dw = synth.DECODE_WORKLOADS[args.decode]
     if args.decode_batch:
@@ -614,6 +807,11 @@ def main(argv=None):
                     help="readings also timed with the per-warp (32-row) vote; '' for none")
     ap.add_argument("--sweep", action="store_true",
                     help="threshold sweep of --prefill (default: the 128K long prefill)")
+    ap.add_argument("--calibrate", action="store_true",
+                    help="calibrate the factors to --targets skip ratios and time them")
+    ap.add_argument("--targets", default="0.25,0.5,0.75")
+    ap.add_argument("--reorder", action="store_true",
+                    help="video prefill in raster vs Hilbert token order")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
@@ -628,6 +826,12 @@ def main(argv=None):
         return
     if args.sweep:
         run_sweep(args)
+        return
+    if args.calibrate:
+        run_calibration(args)
+        return
+    if args.reorder:
+        run_reorder(args)
         return
     run_gpu(args, w, rank, world, local_rank)
 

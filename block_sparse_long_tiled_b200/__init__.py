@@ -26,7 +26,9 @@ SSKIP_OK, SSKIP_ERR_INVALID_ARG, SSKIP_ERR_UNSUPPORTED, SSKIP_ERR_CUDA, SSKIP_ER
 EXPORTS = ("sskip_version", "sskip_status_string", "sskip_device_supported",
            "sskip_attn_prefill", "sskip_attn_prefill_ex", "sskip_attn_prefill_vote",
            "sskip_attn_decode_workspace_size",
-           "sskip_attn_decode", "sskip_attn_decode_ex", "sskip_attn_decode_noalloc",
+           "sskip_attn_decode", "sskip_attn_decode_ex", "sskip_attn_decode_crit",
+           "sskip_attn_decode_noalloc", "sskip_calibrate_factor", "sskip_hilbert3d_order",
+           "sskip_permute_rows",
            "sskip_get_status", "sskip_selftest_watchdog")
 
 # Size of the library's fixed decode scratch (see sskip_attn_decode_noalloc).
@@ -63,7 +65,7 @@ def lib() -> ctypes.CDLL:
         L.sskip_attn_prefill_ex.restype = I
         L.sskip_attn_prefill_ex.argtypes = pre[:-1] + [P, P, P]
         L.sskip_attn_prefill_vote.restype = I
-        L.sskip_attn_prefill_vote.argtypes = pre[:-1] + [I, P, P, P, P]
+        L.sskip_attn_prefill_vote.argtypes = pre[:-1] + [I, P, P, P, P, P]
         L.sskip_attn_decode_workspace_size.restype = Z
         L.sskip_attn_decode_workspace_size.argtypes = [I, I, I, I]
         dec = [P, P, P, P, P, P, I, I, I, I, I, F, F, I, I, P, Z, P]
@@ -71,6 +73,15 @@ def lib() -> ctypes.CDLL:
         L.sskip_attn_decode.argtypes = dec + [P]
         L.sskip_attn_decode_ex.restype = I
         L.sskip_attn_decode_ex.argtypes = dec + [P, P]
+        L.sskip_attn_decode_crit.restype = I
+        L.sskip_attn_decode_crit.argtypes = dec + [P, P, P]
+        D = ctypes.c_double
+        L.sskip_calibrate_factor.restype = I
+        L.sskip_calibrate_factor.argtypes = [P, Z, D, D, P, P, P]
+        L.sskip_hilbert3d_order.restype = I
+        L.sskip_hilbert3d_order.argtypes = [I, I, I, I, P]
+        L.sskip_permute_rows.restype = I
+        L.sskip_permute_rows.argtypes = [P, P, P, ctypes.c_longlong, I, I, I, P]
         L.sskip_attn_decode_noalloc.restype = I
         L.sskip_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, F, I, I, P, P]
         L.sskip_get_status.restype = I
@@ -129,9 +140,10 @@ def sskip_attn_prefill(q, k, v, o, lse, *, causal: bool, sm_scale: float,
 def sskip_attn_prefill_vote(q, k, v, o, lse, *, causal: bool, sm_scale: float,
                             threshold_scale_factor: float, Br: int = 128, Bc: int = 128,
                             vote_rows: int = 32, counts=None, tile_state=None, slice_mask=None,
-                            stream=None) -> None:
+                            tile_crit=None, stream=None) -> None:
     """Marshal the prefill tensors plus vote_rows, counts int64[4] (optional),
-    tile_state and slice_mask uint8 (optional) into sskip_attn_prefill_vote."""
+    tile_state and slice_mask uint8 and tile_crit fp32 (optional) into
+    sskip_attn_prefill_vote."""
     for t in (q, k, v, o):
         _bf16_view(t)
     B, Hq, L, d = q.shape
@@ -140,7 +152,7 @@ def sskip_attn_prefill_vote(q, k, v, o, lse, *, causal: bool, sm_scale: float,
                                        Hkv, L, d, int(bool(causal)), float(sm_scale),
                                        float(threshold_scale_factor), int(Br), int(Bc),
                                        int(vote_rows), _ptr(counts), _ptr(tile_state),
-                                       _ptr(slice_mask), _stream(stream))
+                                       _ptr(slice_mask), _ptr(tile_crit), _stream(stream))
     _check(rc, "sskip_attn_prefill_vote")
 
 
@@ -164,6 +176,38 @@ def sskip_attn_decode(q, kcache, vcache, seqlens, o, lse, *, sm_scale: float,
                                     _ptr(workspace), ws_bytes, _ptr(skip_count), _ptr(tile_state),
                                     _stream(stream))
     _check(rc, "sskip_attn_decode")
+
+
+def sskip_attn_decode_crit(q, kcache, vcache, seqlens, o, lse, *, sm_scale: float,
+                           threshold_scale_factor: float, Bc: int = 64, num_splits: int = 16,
+                           workspace=None, skip_count=None, tile_state=None, tile_crit=None,
+                           stream=None) -> None:
+    """sskip_attn_decode plus the fp32 critical-value record tile_crit
+    [B, Hkv, ceil(Lmax/Bc)] (sskip_attn_decode_crit)."""
+    for t in (q, kcache, vcache, o):
+        _bf16_view(t)
+    B, Hq, d = q.shape
+    Hkv, Lmax = kcache.shape[1], kcache.shape[2]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().sskip_attn_decode_crit(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens),
+                                      _ptr(o), _ptr(lse), B, Hq, Hkv, Lmax, d, float(sm_scale),
+                                      float(threshold_scale_factor), int(Bc), int(num_splits),
+                                      _ptr(workspace), ws_bytes, _ptr(skip_count),
+                                      _ptr(tile_state), _ptr(tile_crit), _stream(stream))
+    _check(rc, "sskip_attn_decode_crit")
+
+
+def sskip_calibrate_factor(tile_crit_host, target_ratio: float, max_factor: float) -> dict:
+    """Marshal a host fp32 critical-value record into sskip_calibrate_factor."""
+    import numpy as np
+    a = np.ascontiguousarray(np.asarray(tile_crit_host, dtype=np.float32)).reshape(-1)
+    f, r = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    v = ctypes.c_longlong(0)
+    rc = lib().sskip_calibrate_factor(a.ctypes.data_as(ctypes.c_void_p), a.size,
+                                      float(target_ratio), float(max_factor), ctypes.byref(f),
+                                      ctypes.byref(r), ctypes.byref(v))
+    _check(rc, "sskip_calibrate_factor")
+    return {"factor": f.value, "achieved_ratio": r.value, "visited": v.value}
 
 
 def sskip_attn_decode_noalloc(q, kcache, vcache, seqlens, o, lse, *, sm_scale: float,
@@ -238,3 +282,85 @@ def decode(q, kcache, vcache, seqlens, *, sm_scale: float, threshold_scale_facto
                       threshold_scale_factor=threshold_scale_factor, Bc=Bc, num_splits=num_splits,
                       workspace=ws, skip_count=counts, tile_state=tiles, stream=stream)
     return {"o": o, "lse": lse, "counts": counts, "tile_state": tiles}
+
+
+def calibrate_prefill(q, k, v, *, causal: bool, sm_scale: float, target_ratio: float,
+                      Br: int = 128, Bc: int = 128, stream=None) -> dict:
+    """One prefill pass (factor 0) with the critical-value record on the GPU,
+    then the host selection of the factor that skips target_ratio of the
+    tiles. Returns factor, achieved_ratio, visited and the record."""
+    B, Hq, L, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+    crit = torch.empty((B, Hq, -(-L // Br), -(-L // Bc)), dtype=torch.float32, device=q.device)
+    sskip_attn_prefill_vote(q, k, v, o, lse, causal=causal, sm_scale=sm_scale,
+                            threshold_scale_factor=0.0, Br=Br, Bc=Bc, vote_rows=Br,
+                            tile_crit=crit, stream=stream)
+    host = crit.cpu().numpy()
+    out = sskip_calibrate_factor(host, target_ratio, float(L))
+    out["tile_crit"] = host
+    return out
+
+
+def calibrate_decode(q, kcache, vcache, seqlens, *, sm_scale: float, target_ratio: float,
+                     Bc: int = 64, num_splits: int = 16, stream=None) -> dict:
+    """Decode counterpart of calibrate_prefill (the cap is the shortest
+    sequence, so every t_b = factor / seqlens[b] stays below 1)."""
+    B, Hq, d = q.shape
+    Hkv, Lmax = kcache.shape[1], kcache.shape[2]
+    o = torch.empty((B, Hq, d), dtype=q.dtype, device=q.device)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws = torch.empty(sskip_attn_decode_workspace_size(B, Hq, d, num_splits), dtype=torch.uint8,
+                     device=q.device)
+    crit = torch.empty((B, Hkv, -(-Lmax // Bc)), dtype=torch.float32, device=q.device)
+    sskip_attn_decode_crit(q, kcache, vcache, seqlens, o, lse, sm_scale=sm_scale,
+                           threshold_scale_factor=0.0, Bc=Bc, num_splits=num_splits,
+                           workspace=ws, tile_crit=crit, stream=stream)
+    host = crit.cpu().numpy()
+    out = sskip_calibrate_factor(host, target_ratio, float(seqlens.min().item()))
+    out["tile_crit"] = host
+    return out
+
+
+def sskip_hilbert3d_order(T: int, H: int, W: int, L: int):
+    """Host int32 numpy [L]: raster index of the token at each position of the
+    3-D Hilbert order (sskip_hilbert3d_order)."""
+    import numpy as np
+    perm = np.empty(L, np.int32)
+    _check(lib().sskip_hilbert3d_order(int(T), int(H), int(W), int(L),
+                                       perm.ctypes.data_as(ctypes.c_void_p)),
+           "sskip_hilbert3d_order")
+    return perm
+
+
+def sskip_permute_rows(src, dst, idx, *, scatter: bool, stream=None) -> None:
+    """Marshal src/dst [..., L, row] (contiguous, same shape) and idx int32 [L]
+    into sskip_permute_rows; n_mats = product of the leading dims."""
+    if src.shape != dst.shape or not (src.is_contiguous() and dst.is_contiguous()):
+        raise ValueError("src and dst must be contiguous and of one shape")
+    L = src.shape[-2]
+    row_bytes = src.shape[-1] * src.element_size()
+    n_mats = src.numel() // (L * src.shape[-1])
+    _check(lib().sskip_permute_rows(_ptr(src), _ptr(dst), _ptr(idx), n_mats, L, row_bytes,
+                                    int(bool(scatter)), _stream(stream)), "sskip_permute_rows")
+
+
+def prefill_reordered(q, k, v, perm, *, sm_scale: float, threshold_scale_factor: float,
+                      Br: int = 128, Bc: int = 128, vote_rows: int | None = None,
+                      stream=None) -> dict:
+    """Non-causal prefill in the token order `perm` (device int32 [L], e.g.
+    the Hilbert order): gather Q, K, V, run the kernel, scatter O and lse back
+    to the original order. Every step runs in the library's kernels."""
+    qp, kp, vp = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    for a, b in ((q, qp), (k, kp), (v, vp)):
+        sskip_permute_rows(a, b, perm, scatter=False, stream=stream)
+    out = prefill(qp, kp, vp, causal=False, sm_scale=sm_scale,
+                  threshold_scale_factor=threshold_scale_factor, Br=Br, Bc=Bc,
+                  vote_rows=vote_rows, stream=stream)
+    o = torch.empty_like(out["o"])
+    lse = torch.empty_like(out["lse"])
+    sskip_permute_rows(out["o"], o, perm, scatter=True, stream=stream)
+    sskip_permute_rows(out["lse"].unsqueeze(-1), lse.unsqueeze(-1), perm, scatter=True,
+                       stream=stream)
+    out.update(o=o, lse=lse)
+    return out

@@ -41,6 +41,7 @@ struct DecodeParams {
   float* lse;                // [B, Hq]
   unsigned long long* counts;  // {skipped, visited} or null
   uint8_t* tile_state;       // [B, Hkv, n_k_max] or null
+  float* tile_crit;          // [B, Hkv, n_k_max] or null: ln of the skipping factor
   int B, Hq, Hkv, Lmax, S, n_k_max;
   float scale_log2;          // sm_scale * log2(e)
   float tsf;                 // threshold_scale_factor
@@ -256,6 +257,17 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       for (int w = 1; w < kDecWarps; ++w) m_loc = fmaxf(m_loc, wm[w]);
       const bool skip =
           __all_sync(0xffffffffu, row_passes_log2(m_loc, m_run, log2_t, t_positive));
+      if (warp == 0 && p.tile_crit) {
+        // Critical factor: the tile is skipped iff ln(tsf) > max over the G
+        // heads of (m_local - m_run) + ln(L_b) (any factor while t_b < 1).
+        float gap = (m_loc == -INFINITY) ? -INFINITY
+                    : (m_run == -INFINITY) ? INFINITY : m_loc - m_run;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) gap = fmaxf(gap, __shfl_xor_sync(0xffffffffu, gap, o));
+        if (lane == 0)
+          p.tile_crit[((size_t)b * p.Hkv + kvh) * p.n_k_max + j0 + t] =
+              gap * 0.69314718055994531f + logf((float)Lb);
+      }
       if (!skip) {
         const float m_new = fmaxf(m_run, m_loc);
         const float a = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);

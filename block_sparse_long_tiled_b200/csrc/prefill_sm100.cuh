@@ -49,6 +49,8 @@ struct PrefillParams {
   unsigned long long* counts;  // {skipped, visited[, slices skipped, slices visited]} or null
   uint8_t* tile_state;         // [B, Hq, n_q, n_k] or null
   uint8_t* slice_mask;         // [B, Hq, n_q, n_k] or null: 0x80 | slices that skipped
+  float* tile_crit;            // [B, Hq, n_q, n_k] or null: ln of the skipping factor
+  float ln_L;                  // ln(L)
   int slice_vote;              // 1: each 32-row warp slice votes alone
   int n_counts;                // 2 or 4 entries in counts
   int B, Hq, Hkv, L, G;
@@ -81,9 +83,16 @@ constexpr int kPfVoteSlots = 4;
 #ifndef SSKIP_PF_NACC
 #define SSKIP_PF_NACC 4       // independent packed accumulators of the row sum
 #endif
-constexpr int kExp2FmaPairsPer8 = SSKIP_PF_FMA_EXP;
+#ifndef SSKIP_PF_FMA_EXP_D64
+#define SSKIP_PF_FMA_EXP_D64 SSKIP_PF_FMA_EXP  // the same, for head dim 64
+#endif
+// At d = 64 a tile's exponentials outweigh its MMAs (16 exp2 per clock per SM
+// on MUFU against 128 x 128 x 64 x 4 FLOP), so part of them may run on the FMA
+// pipe instead; at d = 128 the two are balanced.
+template <int D>
 __device__ __forceinline__ constexpr bool exp2_on_fma(int pair) {
-  return kExp2FmaPairsPer8 > 0 && ((pair & 7) * kExp2FmaPairsPer8) % 8 < kExp2FmaPairsPer8;
+  constexpr int n = D == 64 ? SSKIP_PF_FMA_EXP_D64 : SSKIP_PF_FMA_EXP;
+  return n > 0 && ((pair & 7) * n) % 8 < n;
 }
 // Byte-permute packing rounds each (non-negative) P to bf16 half-up: add half
 // a bf16 unit in the last place to the fp32 bits, keep the top 16 bits.  It
@@ -109,8 +118,9 @@ struct PrefillCfg {
   // dec[2], vote_full[2][VS], vote_empty[2][VS], mma_done
   static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 4 * kPfVoteSlots + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
-  // dec_kept[2], vote_kept[VS][2], warp vote flags [2 wg][2 parity][4], tmem, abort
-  static constexpr int kMiscInts = 2 + 2 * kPfVoteSlots + 16 + 2;
+  // dec_kept[2], vote_kept[VS][2], warp vote flags [2 wg][2 parity][4], tmem, abort,
+  // warp gaps [2 wg][2 parity][4] (fp32)
+  static constexpr int kMiscInts = 2 + 2 * kPfVoteSlots + 16 + 2 + 16;
   static constexpr int kTotal = kMisc + kMiscInts * 4;
   static constexpr int kAlloc = kTotal + 1024;  // room to align the base to 1 KB
   static constexpr int kTmemCols = (2 * BC + 2 * D) <= 256 ? 256 : 512;
@@ -118,7 +128,10 @@ struct PrefillCfg {
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
 
-template <int D, int BR, int BC, bool CAUSAL>
+// EXT = false compiles the plain block vote with the tile_state record only;
+// EXT = true adds the per-warp vote, the slice and critical-value records and
+// the four counters (kept out of the plain kernel, which they slow down).
+template <int D, int BR, int BC, bool CAUSAL, bool EXT>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
@@ -141,6 +154,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   int* wflag = misc + 2 + 2 * VS;            // [2 wg][2 parity][4 warps]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 2 + 2 * VS + 16);
   volatile int* abort_flag = misc + 2 + 2 * VS + 17;
+  float* wgap = reinterpret_cast<float*>(misc + 2 + 2 * VS + 18);  // [2 wg][2 parity][4 warps]
 
   const uint32_t b_qfull = smem_u32(&bars[0]);
   auto b_kfull = [&](int s) { return smem_u32(&bars[1 + s]); };
@@ -442,6 +456,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const bool pass = row_passes_log2(m_loc, m_run, log2_t, t_pos);
       const bool wall = __all_sync(0xffffffffu, !(row_in && gvis) || pass);
       if (lane == 0) wflag[(wg * 2 + (j & 1)) * 4 + wq] = wall ? 1 : 0;
+      if (EXT && p.tile_crit) {
+        // Largest gap m_local - m_run over the warp's valid rows (log2 units).
+        float gap = (!(row_in && gvis) || m_loc == -INFINITY) ? -INFINITY
+                    : (m_run == -INFINITY) ? INFINITY : m_loc - m_run;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) gap = fmaxf(gap, __shfl_xor_sync(0xffffffffu, gap, o));
+        if (lane == 0) wgap[(wg * 2 + (j & 1)) * 4 + wq] = gap;
+      }
       tc_fence_before();
       named_bar_sync(bar_id, 128);
       bool g_kept[NGRP];
@@ -464,11 +486,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           n_skip += all ? 1 : 0;
           const size_t rec = (((size_t)b * p.Hq + hq) * p.n_q + g_tile[g]) * p.n_k + j;
           if (p.tile_state) p.tile_state[rec] = all ? 2 : 1;
-          if (p.slice_mask) p.slice_mask[rec] = uint8_t(0x80u | (p.slice_vote ? bits : (all ? 1u : 0u)));
+          if (EXT && p.slice_mask)
+            p.slice_mask[rec] = uint8_t(0x80u | (p.slice_vote ? bits : (all ? 1u : 0u)));
+          if (EXT && p.tile_crit) {
+            // Skipped iff ln(tsf) > max gap * ln 2 + ln L (for every factor below L).
+            float gm = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < WPG; ++w) gm = fmaxf(gm, wgap[(wg * 2 + (j & 1)) * 4 + g * WPG + w]);
+            p.tile_crit[rec] = gm * 0.69314718055994531f + p.ln_L;
+          }
         }
       }
       // Slice counters: warps holding at least one valid row of a visiting group.
-      if (lane == 0 && gvis && row0 + 128 * wg + wq * 32 < p.L) {
+      if (EXT && lane == 0 && gvis && row0 + 128 * wg + wq * 32 < p.L) {
         ++n_svis;
         n_sskip += wall ? 1 : 0;
       }
@@ -477,7 +507,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (tile_kept) {
         // Block vote: every row of a kept group updates.  Warp vote: only the
         // rows of a warp slice that did not pass.
-        const bool mine = row_in && (p.slice_vote ? (gvis && !wall) : g_kept[grp]);
+        const bool mine = row_in && ((EXT && p.slice_vote) ? (gvis && !wall) : g_kept[grp]);
         float alpha = 1.f;
         bool rescale = false;
         if (mine) {
@@ -508,7 +538,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             tmem_st32(tO + c * 32, w32);
           }
         }
-        if (__all_sync(0xffffffffu, !mine)) {
+        if (EXT && __all_sync(0xffffffffu, !mine)) {
           // No row of this warp takes part (its slice or group skipped the
           // tile, or it is padding): P = 0 without any exponential.
           uint32_t z[32];
@@ -545,14 +575,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int i = 0; i < 32; ++i) {
               const int c = h * 32 + i;
               float p0, p1;
-              if (SSKIP_PF_SCALAR && !exp2_on_fma(c)) {
+              if (SSKIP_PF_SCALAR && !exp2_on_fma<D>(c)) {
                 p0 = ex2_approx(fmaf(sh[2 * c], scale, nref));
                 p1 = ex2_approx(fmaf(sh[2 * c + 1], scale, nref));
                 suma += p0;
                 sumb += p1;
               } else {
                 const uint64_t x2 = ffma2(f2pack(sh[2 * c], sh[2 * c + 1]), scale2, nref2);
-                if (exp2_on_fma(c)) {
+                if (exp2_on_fma<D>(c)) {
                   f2unpack(exp2_fma2(x2), p0, p1);
                 } else {
                   float x0, x1;
@@ -616,12 +646,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (elected && p.counts) {
       atomicAdd(&p.counts[0], (unsigned long long)n_skip);
       atomicAdd(&p.counts[1], (unsigned long long)n_vis);
-      if (p.n_counts == 4 && !p.slice_vote) {  // one slice per block
+      if (EXT && p.n_counts == 4 && !p.slice_vote) {  // one slice per block
         atomicAdd(&p.counts[2], (unsigned long long)n_skip);
         atomicAdd(&p.counts[3], (unsigned long long)n_vis);
       }
     }
-    if (lane == 0 && p.counts && p.n_counts == 4 && p.slice_vote && n_svis > 0) {
+    if (EXT && lane == 0 && p.counts && p.n_counts == 4 && p.slice_vote && n_svis > 0) {
       atomicAdd(&p.counts[2], (unsigned long long)n_sskip);
       atomicAdd(&p.counts[3], (unsigned long long)n_svis);
     }

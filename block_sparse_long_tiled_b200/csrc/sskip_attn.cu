@@ -12,9 +12,12 @@
 #include <mutex>
 #include <set>
 #include <utility>
+#include <algorithm>
+#include <vector>
 
 #include "../../include/sskip_attn.h"
 #include "decode_sm100.cuh"
+#include "permute_sm100.cuh"
 #include "prefill_sm100.cuh"
 
 #define SSKIP_API extern "C" __attribute__((visibility("default")))
@@ -88,10 +91,10 @@ cudaError_t ensure_smem(const void* kernel, int bytes) {
   return e;
 }
 
-template <int D, int BR, int BC, bool CAUSAL>
-int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                   const PrefillParams& p, cudaStream_t st) {
-  auto kernel = prefill_kernel<D, BR, BC, CAUSAL>;
+template <int D, int BR, int BC, bool CAUSAL, bool EXT>
+int launch_prefill_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const PrefillParams& p, cudaStream_t st) {
+  auto kernel = prefill_kernel<D, BR, BC, CAUSAL, EXT>;
   const int smem = PrefillCfg<D, BC>::kAlloc;
   if (ensure_smem(reinterpret_cast<const void*>(kernel), smem) != cudaSuccess)
     return SSKIP_ERR_CUDA;
@@ -111,6 +114,14 @@ int launch_decode(const DecodeParams& p, cudaStream_t st) {
   if (cudaGetLastError() != cudaSuccess) return SSKIP_ERR_CUDA;
   decode_combine_kernel<D><<<(unsigned)(p.B * p.Hq), 128, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? SSKIP_OK : SSKIP_ERR_CUDA;
+}
+
+template <int D, int BR, int BC, bool CAUSAL>
+int launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                   const PrefillParams& p, cudaStream_t st) {
+  const bool ext = p.slice_vote || p.slice_mask || p.tile_crit || p.n_counts == 4;
+  return ext ? launch_prefill_t<D, BR, BC, CAUSAL, true>(mq, mk, mv, p, st)
+             : launch_prefill_t<D, BR, BC, CAUSAL, false>(mq, mk, mv, p, st);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -145,10 +156,11 @@ namespace {
 int prefill_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                  int Hkv, int L, int d, int causal, float sm_scale, float threshold_scale_factor,
                  int Br, int Bc, int vote_rows, unsigned long long* counts, int n_counts,
-                 uint8_t* tile_state, uint8_t* slice_mask, void* stream) {
+                 uint8_t* tile_state, uint8_t* slice_mask, float* tile_crit, void* stream) {
   if (!q || !k || !v || !o || !lse) return SSKIP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(counts) & 7u))
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(counts) & 7u) ||
+      (reinterpret_cast<uintptr_t>(tile_crit) & 3u))
     return SSKIP_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0) return SSKIP_ERR_INVALID_ARG;
   if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SSKIP_ERR_INVALID_ARG;
@@ -176,6 +188,8 @@ int prefill_impl(const void* q, const void* k, const void* v, void* o, float* ls
   p.tile_state = tile_state;
   p.slice_mask = slice_mask;
   p.slice_vote = vote_rows != Br;
+  p.tile_crit = tile_crit;
+  p.ln_L = (float)std::log((double)L);
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.G = Hq / Hkv;
   p.n_q = (L + Br - 1) / Br;
   p.n_k = (L + Bc - 1) / Bc;
@@ -193,6 +207,10 @@ int prefill_impl(const void* q, const void* k, const void* v, void* o, float* ls
     return SSKIP_ERR_CUDA;
   if (slice_mask &&
       cudaMemsetAsync(slice_mask, 0, (size_t)B * Hq * p.n_q * p.n_k, st) != cudaSuccess)
+    return SSKIP_ERR_CUDA;
+  // 0xFF bytes are a NaN: tiles a call never visits stay NaN.
+  if (tile_crit &&
+      cudaMemsetAsync(tile_crit, 0xFF, (size_t)B * Hq * p.n_q * p.n_k * 4, st) != cudaSuccess)
     return SSKIP_ERR_CUDA;
 
   const bool c = causal != 0;
@@ -215,16 +233,17 @@ SSKIP_API int sskip_attn_prefill_ex(const void* q, const void* k, const void* v,
                                     unsigned long long* skip_count, uint8_t* tile_state,
                                     void* stream) {
   return prefill_impl(q, k, v, o, lse, B, Hq, Hkv, L, d, causal, sm_scale, threshold_scale_factor,
-                      Br, Bc, Br, skip_count, 2, tile_state, nullptr, stream);
+                      Br, Bc, Br, skip_count, 2, tile_state, nullptr, nullptr, stream);
 }
 
 SSKIP_API int sskip_attn_prefill_vote(const void* q, const void* k, const void* v, void* o,
                                       float* lse, int B, int Hq, int Hkv, int L, int d, int causal,
                                       float sm_scale, float threshold_scale_factor, int Br, int Bc,
                                       int vote_rows, unsigned long long* counts,
-                                      uint8_t* tile_state, uint8_t* slice_mask, void* stream) {
+                                      uint8_t* tile_state, uint8_t* slice_mask, float* tile_crit,
+                                      void* stream) {
   return prefill_impl(q, k, v, o, lse, B, Hq, Hkv, L, d, causal, sm_scale, threshold_scale_factor,
-                      Br, Bc, vote_rows, counts, 4, tile_state, slice_mask, stream);
+                      Br, Bc, vote_rows, counts, 4, tile_state, slice_mask, tile_crit, stream);
 }
 
 SSKIP_API int sskip_attn_prefill(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -241,18 +260,20 @@ SSKIP_API size_t sskip_attn_decode_workspace_size(int B, int Hq, int d, int num_
   return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
 }
 
-SSKIP_API int sskip_attn_decode_ex(const void* q, const void* kcache, const void* vcache,
-                                   const int* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
-                                   int Lmax, int d, float sm_scale, float threshold_scale_factor,
-                                   int Bc, int num_splits, void* workspace, size_t workspace_bytes,
-                                   unsigned long long* skip_count, uint8_t* tile_state,
-                                   void* stream) {
+namespace sskip {
+namespace {
+
+int decode_impl(const void* q, const void* kcache, const void* vcache, const int* seqlens, void* o,
+                float* lse, int B, int Hq, int Hkv, int Lmax, int d, float sm_scale,
+                float threshold_scale_factor, int Bc, int num_splits, void* workspace,
+                size_t workspace_bytes, unsigned long long* skip_count, uint8_t* tile_state,
+                float* tile_crit, void* stream) {
   if (!q || !kcache || !vcache || !seqlens || !o || !lse || !workspace)
     return SSKIP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
       (reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
-      (reinterpret_cast<uintptr_t>(skip_count) & 7u))
+      (reinterpret_cast<uintptr_t>(skip_count) & 7u) || (reinterpret_cast<uintptr_t>(tile_crit) & 3u))
     return SSKIP_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || Lmax < 1 || Hq % Hkv != 0 || num_splits < 1)
     return SSKIP_ERR_INVALID_ARG;
@@ -280,6 +301,7 @@ SSKIP_API int sskip_attn_decode_ex(const void* q, const void* kcache, const void
   p.lse = lse;
   p.counts = skip_count;
   p.tile_state = tile_state;
+  p.tile_crit = tile_crit;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lmax = Lmax; p.S = num_splits;
   p.n_k_max = (Lmax + kDecBc - 1) / kDecBc;
   p.scale_log2 = (float)((double)sm_scale * 1.4426950408889634);
@@ -289,6 +311,10 @@ SSKIP_API int sskip_attn_decode_ex(const void* q, const void* kcache, const void
     return SSKIP_ERR_CUDA;
   if (tile_state &&
       cudaMemsetAsync(tile_state, 0, (size_t)B * Hkv * p.n_k_max, st) != cudaSuccess)
+    return SSKIP_ERR_CUDA;
+  // 0xFF bytes are a NaN: tiles a call never visits stay NaN.
+  if (tile_crit &&
+      cudaMemsetAsync(tile_crit, 0xFF, (size_t)B * Hkv * p.n_k_max * 4, st) != cudaSuccess)
     return SSKIP_ERR_CUDA;
 
   if (d == 128) {
@@ -305,6 +331,32 @@ SSKIP_API int sskip_attn_decode_ex(const void* q, const void* kcache, const void
     case 4: return launch_decode<64, 4>(p, st);
     default: return launch_decode<64, 8>(p, st);
   }
+}
+
+}  // namespace
+}  // namespace sskip
+
+SSKIP_API int sskip_attn_decode_ex(const void* q, const void* kcache, const void* vcache,
+                                   const int* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
+                                   int Lmax, int d, float sm_scale, float threshold_scale_factor,
+                                   int Bc, int num_splits, void* workspace, size_t workspace_bytes,
+                                   unsigned long long* skip_count, uint8_t* tile_state,
+                                   void* stream) {
+  return decode_impl(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Lmax, d, sm_scale,
+                     threshold_scale_factor, Bc, num_splits, workspace, workspace_bytes,
+                     skip_count, tile_state, nullptr, stream);
+}
+
+SSKIP_API int sskip_attn_decode_crit(const void* q, const void* kcache, const void* vcache,
+                                     const int* seqlens, void* o, float* lse, int B, int Hq,
+                                     int Hkv, int Lmax, int d, float sm_scale,
+                                     float threshold_scale_factor, int Bc, int num_splits,
+                                     void* workspace, size_t workspace_bytes,
+                                     unsigned long long* skip_count, uint8_t* tile_state,
+                                     float* tile_crit, void* stream) {
+  return decode_impl(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Lmax, d, sm_scale,
+                     threshold_scale_factor, Bc, num_splits, workspace, workspace_bytes,
+                     skip_count, tile_state, tile_crit, stream);
 }
 
 SSKIP_API int sskip_attn_decode(const void* q, const void* kcache, const void* vcache,
@@ -383,4 +435,143 @@ SSKIP_API int sskip_attn_decode_noalloc(const void* q, const void* kcache, const
                               threshold_scale_factor, Bc, num_splits, scratch,
                               (size_t)SSKIP_DECODE_NOALLOC_SCRATCH_BYTES, skip_count, nullptr,
                               stream);
+}
+
+// ---------------------------------------------------------------------------
+// Threshold calibration: choose the factor that skips a target share of tiles.
+//
+// While t < 1 no passing row can raise its running maximum, so the running
+// maximum is the prefix maximum of the local maxima whatever was skipped and a
+// tile is skipped exactly when ln(factor) exceeds its critical value
+// c = max_rows (m_local - m_run) + ln L.  The skip count is therefore the
+// number of critical values below ln(factor), and the factor for a target
+// count k lies just above the k-th smallest critical value.  The factor is
+// placed halfway (in ln) between that value and the next larger one, away
+// from both decision boundaries.
+SSKIP_API int sskip_calibrate_factor(const float* tile_crit, size_t n, double target_ratio,
+                                     double max_factor, double* factor, double* achieved_ratio,
+                                     long long* visited_out) {
+  if (!tile_crit || !factor || !(target_ratio >= 0.0) || !(target_ratio <= 1.0))
+    return SSKIP_ERR_INVALID_ARG;
+  std::vector<float> c;
+  c.reserve(n);
+  long long visited = 0;
+  for (size_t i = 0; i < n; ++i) {
+    const float x = tile_crit[i];
+    if (x != x) continue;  // not visited
+    ++visited;
+    if (x < INFINITY) c.push_back(x);
+  }
+  if (visited_out) *visited_out = visited;
+  if (visited == 0) return SSKIP_ERR_INVALID_ARG;
+  const long long k = std::min<long long>(
+      visited, std::max<long long>(0, (long long)std::ceil(target_ratio * (double)visited - 1e-9)));
+  const double ln_max = max_factor > 0.0 ? std::log(max_factor) : INFINITY;
+  if (k == 0) {
+    *factor = 0.0;  // factor 0 skips nothing
+    if (achieved_ratio) *achieved_ratio = 0.0;
+    return SSKIP_OK;
+  }
+  if (k > (long long)c.size()) return SSKIP_ERR_UNSUPPORTED;
+  std::nth_element(c.begin(), c.begin() + (k - 1), c.end());
+  const double ck = c[k - 1];
+  double cn = INFINITY;  // next larger critical value
+  for (size_t i = (size_t)k; i < c.size(); ++i)
+    if (c[i] > ck && c[i] < cn) cn = c[i];
+  if (!(ck < ln_max)) return SSKIP_ERR_UNSUPPORTED;  // would need t >= 1
+  const double hi = std::min(cn, ln_max);
+  double ln_f;
+  if (std::isinf(ck)) ln_f = std::isinf(hi) ? 0.0 : hi - 1.0;  // ck = -inf: any factor > 0
+  else ln_f = std::isinf(hi) ? ck + 1.0 : 0.5 * (ck + hi);
+  *factor = std::exp(ln_f);
+  if (achieved_ratio) {
+    long long below = 0;
+    for (float x : c) below += (double)x < ln_f;
+    *achieved_ratio = (double)below / (double)visited;
+  }
+  return SSKIP_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Token reordering (SpargeAttn article, "Hilbert 曲线置换").
+namespace sskip {
+namespace {
+
+// Position of a 3-D point on the Hilbert curve of side 2^bits, by John
+// Skilling's method ("Programming the Hilbert curve", AIP Conf. Proc. 707,
+// 2004): the axes are turned into the transposed index by undoing the curve's
+// reflections and exchanges from the top bit down plus a Gray code, and the
+// transposed index is read out bit plane by bit plane.
+uint64_t hilbert3(uint32_t a0, uint32_t a1, uint32_t a2, int bits) {
+  uint32_t ax[3] = {a0, a1, a2};
+  for (uint32_t q = 1u << (bits - 1); q > 1; q >>= 1) {
+    const uint32_t low = q - 1;
+    for (int d = 0; d < 3; ++d) {
+      if (ax[d] & q) {
+        ax[0] ^= low;
+      } else {
+        const uint32_t sw = (ax[0] ^ ax[d]) & low;
+        ax[0] ^= sw;
+        ax[d] ^= sw;
+      }
+    }
+  }
+  ax[1] ^= ax[0];
+  ax[2] ^= ax[1];
+  uint32_t flip = 0;
+  for (uint32_t q = 1u << (bits - 1); q > 1; q >>= 1)
+    if (ax[2] & q) flip ^= q - 1;
+  for (int d = 0; d < 3; ++d) ax[d] ^= flip;
+  uint64_t h = 0;
+  for (int bit = bits - 1; bit >= 0; --bit)
+    for (int d = 0; d < 3; ++d) h = (h << 1) | ((ax[d] >> bit) & 1u);
+  return h;
+}
+
+}  // namespace
+}  // namespace sskip
+
+SSKIP_API int sskip_hilbert3d_order(int T, int H, int W, int L, int32_t* perm) {
+  if (!perm || T < 1 || H < 1 || W < 1 || L < 1 || (long long)T * H * W < L)
+    return SSKIP_ERR_INVALID_ARG;
+  int bits = 1;
+  while ((1 << bits) < std::max(T, std::max(H, W))) ++bits;
+  if (bits > 20) return SSKIP_ERR_UNSUPPORTED;
+  std::vector<std::pair<uint64_t, int32_t>> key(L);
+  for (int i = 0; i < L; ++i) {
+    const int t = i / (H * W), h = (i / W) % H, w = i % W;  // t-major raster
+    key[i] = {hilbert3((uint32_t)t, (uint32_t)h, (uint32_t)w, bits), i};
+  }
+  std::sort(key.begin(), key.end());  // keys are distinct: a bijection of the cube
+  for (int s = 0; s < L; ++s) perm[s] = key[s].second;
+  return SSKIP_OK;
+}
+
+SSKIP_API int sskip_permute_rows(const void* src, void* dst, const int32_t* idx, long long n_mats,
+                                 int L, int row_bytes, int scatter, void* stream) {
+  if (!src || !dst || !idx || src == dst || n_mats < 1 || L < 1 || row_bytes < 4 ||
+      row_bytes % 4 != 0 || (reinterpret_cast<uintptr_t>(idx) & 3u))
+    return SSKIP_ERR_INVALID_ARG;
+  const bool v16 = row_bytes % 16 == 0 && aligned16(src) && aligned16(dst);
+  if (!v16 && ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 3u))
+    return SSKIP_ERR_INVALID_ARG;
+  const int cpr = row_bytes / (v16 ? 16 : 4);
+  const long long total = n_mats * (long long)L * cpr;
+  int sms = 148;
+  {
+    int dev = current_device();
+    if (dev >= 0) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const long long want = (total + 255) / 256;
+  const unsigned grid = (unsigned)std::max<long long>(1, std::min<long long>(want, (long long)sms * 8));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (v16)
+    permute_rows_kernel<uint4><<<grid, 256, 0, st>>>(static_cast<const uint4*>(src),
+                                                     static_cast<uint4*>(dst), idx, n_mats, L, cpr,
+                                                     scatter != 0);
+  else
+    permute_rows_kernel<uint32_t><<<grid, 256, 0, st>>>(static_cast<const uint32_t*>(src),
+                                                         static_cast<uint32_t*>(dst), idx, n_mats,
+                                                         L, cpr, scatter != 0);
+  return cudaGetLastError() == cudaSuccess ? SSKIP_OK : SSKIP_ERR_CUDA;
 }

@@ -120,12 +120,21 @@ int sskip_attn_prefill_ex(const void* q, const void* k, const void* v, void* o, 
  *     0 = tile not visited, else 0x80 | bit s set when slice s (rows
  *     [s * vote_rows, (s + 1) * vote_rows) of the query tile) skipped it.  A
  *     slice with no row < L passes vacuously (its bit is set).
+ *   tile_crit: optional device fp32 [B, Hq, ceil(L/Br), ceil(L/Bc)], 4-byte
+ *     aligned: per visited tile its critical value, the natural log of the
+ *     smallest threshold_scale_factor that skips it under the block vote,
+ *     c = max over valid rows (m_local - m_run) + ln L, with m_run the running
+ *     maximum before the tile; +inf for a tile no factor skips (the first
+ *     tile of a row), NaN where the tile is not visited.  While t < 1 the
+ *     running maximum does not depend on what was skipped, so the record is
+ *     the same at every factor below L and the call skips a tile exactly when
+ *     ln(threshold_scale_factor) > c.  The input of sskip_calibrate_factor.
  */
 int sskip_attn_prefill_vote(const void* q, const void* k, const void* v, void* o, float* lse,
                             int B, int Hq, int Hkv, int L, int d, int causal, float sm_scale,
                             float threshold_scale_factor, int Br, int Bc, int vote_rows,
                             unsigned long long* counts, uint8_t* tile_state,
-                            uint8_t* slice_mask, void* stream);
+                            uint8_t* slice_mask, float* tile_crit, void* stream);
 
 /*
  * Decode: one new query token per sequence against a contiguous KV cache,
@@ -172,6 +181,47 @@ int sskip_attn_decode_ex(const void* q, const void* kcache, const void* vcache,
                          unsigned long long* skip_count, uint8_t* tile_state, void* stream);
 
 /*
+ * Same as sskip_attn_decode_ex, plus an optional record of each decode tile's
+ * critical value (see sskip_attn_prefill_vote): tile_crit, device fp32
+ * [B, Hkv, ceil(Lmax/Bc)], 4-byte aligned; c = max over the G heads of
+ * (m_local - m_run) + ln(seqlens[b]) with m_run the running maximum of the
+ * tile's split (+inf for the first tile of a split), NaN for tiles past
+ * seqlens[b].  The call skips a tile exactly when ln(factor) > c while
+ * factor < seqlens[b].
+ */
+int sskip_attn_decode_crit(const void* q, const void* kcache, const void* vcache,
+                           const int* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
+                           int Lmax, int d, float sm_scale, float threshold_scale_factor, int Bc,
+                           int num_splits, void* workspace, size_t workspace_bytes,
+                           unsigned long long* skip_count, uint8_t* tile_state, float* tile_crit,
+                           void* stream);
+
+/*
+ * Threshold calibration (the Model Optimizer tutorial's step 4 and the
+ * TensorRT-LLM article's closing "target sparsity in, threshold out" goal):
+ * pick the threshold_scale_factor that skips target_ratio of the visited
+ * tiles, from a tile_crit record taken on calibration inputs.  HOST memory:
+ * tile_crit is a host copy of the record (n floats, NaN = not visited).
+ *
+ *   k = ceil(target_ratio * visited) tiles must be skipped; the factor is
+ *   placed halfway, in natural log, between the k-th smallest critical value
+ *   and the next larger one (capped by max_factor), so every tile whose
+ *   critical value is at most the k-th is skipped and no other.
+ *   max_factor: the smallest context length of the data (the factor must keep
+ *     t = factor / L < 1 for the record to hold); <= 0 disables the cap.
+ *   factor (out): the factor; 0 when target_ratio rounds to zero tiles.
+ *   achieved_ratio (out, may be NULL): skipped / visited at that factor
+ *     (>= target_ratio; above it only when critical values tie).
+ *   visited_out (out, may be NULL): the number of visited tiles.
+ *   Returns SSKIP_ERR_UNSUPPORTED when the target cannot be reached below
+ *   max_factor, SSKIP_ERR_INVALID_ARG for a bad argument or an empty record.
+ *   Pure host code: no CUDA call.
+ */
+int sskip_calibrate_factor(const float* tile_crit, size_t n, double target_ratio,
+                           double max_factor, double* factor, double* achieved_ratio,
+                           long long* visited_out);
+
+/*
  * Decode for callers that cannot allocate device memory.  The paper has no
  * counterpart: this is a deployment variant of sskip_attn_decode.
  *
@@ -206,6 +256,37 @@ int sskip_attn_decode_noalloc(const void* q, const void* kcache, const void* vca
                               int B, int Hq, int Hkv, int Lmax, int d, float sm_scale,
                               float threshold_scale_factor, int Bc, int num_splits,
                               unsigned long long* skip_count, void* stream);
+
+/*
+ * Token reordering along a 3-D Hilbert curve (SpargeAttn article, "Hilbert
+ * 曲线置换": the T x H x W visual tokens are laid out along a Hilbert curve
+ * before attention so that the tokens of one tile form a compact 3-D region,
+ * which raises the share of tiles that can be skipped).
+ *
+ * sskip_hilbert3d_order: HOST call, no CUDA.  For the first L tokens of the
+ * t-major raster of a T x H x W grid (token i at t = i / (H W),
+ * h = (i / W) % H, w = i % W), writes perm[s] (host int32 [L]) = the raster
+ * index of the token at position s of the Hilbert order: tokens sorted by
+ * their position on the Hilbert curve of the smallest 2^b cube holding the
+ * grid (John Skilling's index; points outside the grid are absent).
+ * Requires L <= T H W.
+ */
+int sskip_hilbert3d_order(int T, int H, int W, int L, int32_t* perm);
+
+/*
+ * sskip_permute_rows: reorders whole rows of n_mats consecutive [L, row]
+ * matrices (device memory, row = row_bytes bytes, a multiple of 4):
+ *   scatter = 0 (gather):  dst[m, i, :] = src[m, idx[i], :]
+ *   scatter = 1 (inverse): dst[m, idx[i], :] = src[m, i, :]
+ * idx: device int32 [L], a permutation of 0 .. L-1; an index outside it is
+ * latched as SSKIP_ERR_INVALID_ARG in the device status word and that row is
+ * not touched.  src and dst must not overlap.  16-byte rows use 16-byte
+ * accesses (pointers then 16-byte aligned), others 4-byte ones.  With perm
+ * from sskip_hilbert3d_order: gather Q, K, V [B, H, L, d] into Hilbert order
+ * (n_mats = B H), run a non-causal prefill, scatter O and lse back.
+ */
+int sskip_permute_rows(const void* src, void* dst, const int32_t* idx, long long n_mats, int L,
+                       int row_bytes, int scatter, void* stream);
 
 /*
  * Synchronises `stream`, then returns and clears the current device's status
