@@ -773,6 +773,75 @@ def run_reorder(args):
                       "runs": rows}), flush=True)
 
 
+def run_step_bench(args):
+    """One serving step (prefill + decode of one layer, factors 1000 / 500 by
+    phase) through sskip_attn_step: eager launches and the same step replayed
+    from a CUDA graph."""
+    import torch
+    import block_sparse_long_tiled_b200 as sk
+    dev = torch.device("cuda", 0)
+    w = synth.PREFILL_WORKLOADS[args.prefill]
+    dw = decode_workload(args)
+    td = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev).view(
+        torch.bfloat16)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    x = synth.prefill_inputs(w, args.reading)
+    P = {"q": td(x["q"]), "k": td(x["k"]), "v": td(x["v"])}
+    del x
+    P["o"] = torch.empty_like(P["q"])
+    P["lse"] = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
+    P["count"] = torch.zeros(2, dtype=torch.int64, device=dev)
+    dx = synth.decode_inputs(dw, args.reading)
+    D = {"q": td(dx["q"]), "kcache": td(dx["kcache"]), "vcache": td(dx["vcache"]),
+         "seqlens": torch.from_numpy(dx["seqlens"]).to(dev)}
+    del dx
+    D["o"] = torch.empty((dw.B, dw.Hq, dw.d), dtype=torch.bfloat16, device=dev)
+    D["lse"] = torch.empty((dw.B, dw.Hq), dtype=torch.float32, device=dev)
+    D["workspace"] = torch.empty(sk.sskip_attn_decode_workspace_size(dw.B, dw.Hq, dw.d,
+                                                                     dw.num_splits),
+                                 dtype=torch.uint8, device=dev)
+    D["count"] = torch.zeros(2, dtype=torch.int64, device=dev)
+    factors = {"prefill": w.tsf, "decode": dw.tsf}
+
+    def step():
+        sk.sskip_attn_step(threshold_scale_factor=factors, sm_scale=w.scale, prefill=P,
+                           decode=D, Br=w.Br, Bc=w.Bc, causal=w.causal,
+                           num_splits=dw.num_splits)
+
+    def time_it(fn):
+        ts = []
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ts.append(a.elapsed_time(b))
+        return float(np.median(ts))
+
+    step()
+    torch.cuda.synchronize()
+    eager = time_it(step)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.current_stream().wait_stream(s)
+    with torch.cuda.graph(g):
+        step()
+    graph = time_it(g.replay)
+    assert sk.sskip_get_status() == sk.SSKIP_OK
+    cp, cd = P["count"].cpu().tolist(), D["count"].cpu().tolist()
+    print(json.dumps({"step": f"{w.name} + {dw.name}", "reading": args.reading,
+                      "threshold_scale_factor": factors, "ms_eager": eager, "ms_graph": graph,
+                      "prefill_skip_fraction": cp[0] / cp[1],
+                      "decode_skip_fraction": cd[0] / cd[1], "launches": 3}), flush=True)
+    del g
+
+
 def decode_workload(args):
     dw = synth.DECODE_WORKLOADS[args.decode]
     if args.decode_batch:
@@ -812,6 +881,8 @@ def main(argv=None):
     ap.add_argument("--targets", default="0.25,0.5,0.75")
     ap.add_argument("--reorder", action="store_true",
                     help="video prefill in raster vs Hilbert token order")
+    ap.add_argument("--step", action="store_true",
+                    help="one serving step (prefill + decode, factor per phase), eager and graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
@@ -832,6 +903,9 @@ def main(argv=None):
         return
     if args.reorder:
         run_reorder(args)
+        return
+    if args.step:
+        run_step_bench(args)
         return
     run_gpu(args, w, rank, world, local_rank)
 

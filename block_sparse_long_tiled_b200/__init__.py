@@ -28,7 +28,7 @@ EXPORTS = ("sskip_version", "sskip_status_string", "sskip_device_supported",
            "sskip_attn_decode_workspace_size",
            "sskip_attn_decode", "sskip_attn_decode_ex", "sskip_attn_decode_crit",
            "sskip_attn_decode_noalloc", "sskip_calibrate_factor", "sskip_hilbert3d_order",
-           "sskip_permute_rows",
+           "sskip_permute_rows", "sskip_attn_step",
            "sskip_get_status", "sskip_selftest_watchdog")
 
 # Size of the library's fixed decode scratch (see sskip_attn_decode_noalloc).
@@ -82,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.sskip_hilbert3d_order.argtypes = [I, I, I, I, P]
         L.sskip_permute_rows.restype = I
         L.sskip_permute_rows.argtypes = [P, P, P, ctypes.c_longlong, I, I, I, P]
+        L.sskip_attn_step.restype = I
+        L.sskip_attn_step.argtypes = ([P, P, P, P, P, I, I, I, I, I, P] +
+                                      [P, P, P, P, P, P, I, I, I, P, Z, P] +
+                                      [I, I, I, F, F, F, P])
         L.sskip_attn_decode_noalloc.restype = I
         L.sskip_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, F, I, I, P, P]
         L.sskip_get_status.restype = I
@@ -347,16 +351,17 @@ def sskip_permute_rows(src, dst, idx, *, scatter: bool, stream=None) -> None:
 
 def prefill_reordered(q, k, v, perm, *, sm_scale: float, threshold_scale_factor: float,
                       Br: int = 128, Bc: int = 128, vote_rows: int | None = None,
-                      stream=None) -> dict:
+                      with_tiles: bool = False, stream=None) -> dict:
     """Non-causal prefill in the token order `perm` (device int32 [L], e.g.
     the Hilbert order): gather Q, K, V, run the kernel, scatter O and lse back
-    to the original order. Every step runs in the library's kernels."""
+    to the original order. Every step runs in the library's kernels; the tile
+    record, if asked for, is in the reordered frame."""
     qp, kp, vp = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     for a, b in ((q, qp), (k, kp), (v, vp)):
         sskip_permute_rows(a, b, perm, scatter=False, stream=stream)
     out = prefill(qp, kp, vp, causal=False, sm_scale=sm_scale,
                   threshold_scale_factor=threshold_scale_factor, Br=Br, Bc=Bc,
-                  vote_rows=vote_rows, stream=stream)
+                  with_tiles=with_tiles, vote_rows=vote_rows, stream=stream)
     o = torch.empty_like(out["o"])
     lse = torch.empty_like(out["lse"])
     sskip_permute_rows(out["o"], o, perm, scatter=True, stream=stream)
@@ -364,3 +369,61 @@ def prefill_reordered(q, k, v, perm, *, sm_scale: float, threshold_scale_factor:
                        stream=stream)
     out.update(o=o, lse=lse)
     return out
+
+
+def phase_factors(threshold_scale_factor) -> tuple[float, float]:
+    """(prefill, decode) factors from one number or a {"prefill", "decode"}
+    mapping, the two forms the TensorRT-LLM configuration accepts."""
+    if isinstance(threshold_scale_factor, dict):
+        extra = set(threshold_scale_factor) - {"prefill", "decode"}
+        if extra or len(threshold_scale_factor) != 2:
+            raise ValueError("threshold_scale_factor needs exactly the keys 'prefill' and 'decode'")
+        return float(threshold_scale_factor["prefill"]), float(threshold_scale_factor["decode"])
+    f = float(threshold_scale_factor)
+    return f, f
+
+
+def sskip_attn_step(*, threshold_scale_factor, sm_scale: float, prefill=None, decode=None,
+                    Br: int = 128, Bc: int = 128, causal: bool = True, num_splits: int = 16,
+                    stream=None) -> None:
+    """Marshal one serving step into sskip_attn_step.
+
+    prefill: dict q, k, v, o, lse (and optional count int64[2]) or None;
+    decode: dict q, kcache, vcache, seqlens, o, lse, workspace (optional count)
+    or None; threshold_scale_factor: a number or {"prefill": a, "decode": b}."""
+    tp, td = phase_factors(threshold_scale_factor)
+    if prefill is None and decode is None:
+        raise ValueError("a step needs a prefill or a decode batch")
+    ref = (prefill or decode)["q"]
+    Hq = ref.shape[1]
+    d = ref.shape[-1]
+    if prefill is not None:
+        for n in ("q", "k", "v", "o"):
+            _bf16_view(prefill[n])
+        Bp, _, L, _ = prefill["q"].shape
+        Hkv = prefill["k"].shape[1]
+    else:
+        Bp, L = 0, 0
+    if decode is not None:
+        for n in ("q", "kcache", "vcache", "o"):
+            _bf16_view(decode[n])
+        Bd = decode["q"].shape[0]
+        Hkv_d, Lmax = decode["kcache"].shape[1], decode["kcache"].shape[2]
+        if prefill is not None and (Hkv_d != Hkv or decode["q"].shape[1] != Hq
+                                    or decode["q"].shape[-1] != d):
+            raise ValueError("both phases must come from one layer (Hq, Hkv, d)")
+        Hkv = Hkv_d
+        ws = decode["workspace"]
+        ws_bytes = ws.numel() * ws.element_size()
+    else:
+        Bd, Lmax, ws, ws_bytes = 0, 0, None, 0
+    P = prefill or {}
+    D = decode or {}
+    rc = lib().sskip_attn_step(_ptr(P.get("q")), _ptr(P.get("k")), _ptr(P.get("v")),
+                               _ptr(P.get("o")), _ptr(P.get("lse")), Bp, L, int(bool(causal)),
+                               int(Br), int(Bc), _ptr(P.get("count")), _ptr(D.get("q")),
+                               _ptr(D.get("kcache")), _ptr(D.get("vcache")),
+                               _ptr(D.get("seqlens")), _ptr(D.get("o")), _ptr(D.get("lse")), Bd,
+                               Lmax, int(num_splits), _ptr(ws), ws_bytes, _ptr(D.get("count")),
+                               Hq, Hkv, d, float(sm_scale), tp, td, _stream(stream))
+    _check(rc, "sskip_attn_step")

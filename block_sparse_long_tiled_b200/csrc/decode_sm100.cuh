@@ -112,8 +112,16 @@ __device__ __forceinline__ float transpose_reduce8(const float (&acc)[G], int su
   return v[0];
 }
 
+// CRIT = true adds the critical-value record; the plain kernel is built
+// without it (the extra branch in the tile loop costs time even when off).
+// Eight heads at d = 128 keep 128 registers of q and 32 of accumulators per
+// thread, more than two CTAs per SM leave (128); they run one CTA per SM.
 template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const DecodeParams p) {
+constexpr int dec_ctas_per_sm() { return (G * D > 512) ? 1 : 2; }
+
+template <int D, int G, bool CRIT>
+__global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
+    decode_split_kernel(const DecodeParams p) {
   using L = DecodeSmem<D, G>;
   constexpr int PPL = D / 64;        // 16-byte pieces per lane per key (8 lanes per key)
   constexpr int EPL = D / 32;        // P.V output elements per lane
@@ -257,7 +265,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       for (int w = 1; w < kDecWarps; ++w) m_loc = fmaxf(m_loc, wm[w]);
       const bool skip =
           __all_sync(0xffffffffu, row_passes_log2(m_loc, m_run, log2_t, t_positive));
-      if (warp == 0 && p.tile_crit) {
+      if (CRIT && warp == 0) {
         // Critical factor: the tile is skipped iff ln(tsf) > max over the G
         // heads of (m_local - m_run) + ln(L_b) (any factor while t_b < 1).
         float gap = (m_loc == -INFINITY) ? -INFINITY

@@ -105,7 +105,7 @@ int launch_prefill_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 
 template <int D, int G>
 int launch_decode(const DecodeParams& p, cudaStream_t st) {
-  auto kernel = decode_split_kernel<D, G>;
+  auto kernel = p.tile_crit ? decode_split_kernel<D, G, true> : decode_split_kernel<D, G, false>;
   const int smem = DecodeSmem<D, G>::kTotal;
   if (ensure_smem(reinterpret_cast<const void*>(kernel), smem) != cudaSuccess)
     return SSKIP_ERR_CUDA;
@@ -574,4 +574,28 @@ SSKIP_API int sskip_permute_rows(const void* src, void* dst, const int32_t* idx,
                                                          static_cast<uint32_t*>(dst), idx, n_mats,
                                                          L, cpr, scatter != 0);
   return cudaGetLastError() == cudaSuccess ? SSKIP_OK : SSKIP_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// One serving step with a factor per phase (TensorRT-LLM article, "实战演练":
+// threshold_scale_factor may be one number or a {prefill, decode} pair).
+SSKIP_API int sskip_attn_step(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int Bp, int L, int causal, int Br, int Bc,
+                              unsigned long long* prefill_count, const void* dq,
+                              const void* kcache, const void* vcache, const int* seqlens,
+                              void* dout, float* dlse, int Bd, int Lmax, int num_splits,
+                              void* workspace, size_t workspace_bytes,
+                              unsigned long long* decode_count, int Hq, int Hkv, int d,
+                              float sm_scale, float tsf_prefill, float tsf_decode, void* stream) {
+  if (Bp < 0 || Bd < 0 || Bp + Bd == 0) return SSKIP_ERR_INVALID_ARG;
+  if (Bp > 0) {
+    const int rc = sskip_attn_prefill_ex(q, k, v, o, lse, Bp, Hq, Hkv, L, d, causal, sm_scale,
+                                         tsf_prefill, Br, Bc, prefill_count, nullptr, stream);
+    if (rc != SSKIP_OK) return rc;
+  }
+  if (Bd > 0)
+    return sskip_attn_decode_ex(dq, kcache, vcache, seqlens, dout, dlse, Bd, Hq, Hkv, Lmax, d,
+                                sm_scale, tsf_decode, kDecBc, num_splits, workspace,
+                                workspace_bytes, decode_count, nullptr, stream);
+  return SSKIP_OK;
 }

@@ -258,6 +258,31 @@ int sskip_attn_decode_noalloc(const void* q, const void* kcache, const void* vca
                               unsigned long long* skip_count, void* stream);
 
 /*
+ * One serving step of one attention layer with a factor per phase: the
+ * TensorRT-LLM article ("实战演练") lets threshold_scale_factor be a single
+ * number or a {prefill: 1000, decode: 500} pair, each divided by its own
+ * context length.  The step runs, in this order on `stream`:
+ *   - the prefill of Bp whole sequences of length L (skipped when Bp = 0),
+ *     exactly sskip_attn_prefill_ex(q, k, v, o, lse, Bp, Hq, Hkv, L, d, causal,
+ *     sm_scale, tsf_prefill, Br, Bc, prefill_count, NULL, stream), so
+ *     t = tsf_prefill / L;
+ *   - the decode of Bd sequences against their caches (skipped when Bd = 0),
+ *     exactly sskip_attn_decode_ex(dq, kcache, vcache, seqlens, dout, dlse, Bd,
+ *     Hq, Hkv, Lmax, d, sm_scale, tsf_decode, 64, num_splits, workspace,
+ *     workspace_bytes, decode_count, NULL, stream), so t_b = tsf_decode /
+ *     seqlens[b].
+ * Hq, Hkv, d and sm_scale are the layer's and shared by both phases.  Returns
+ * the first failing status (the decode is not enqueued after a prefill
+ * error).  Bp = Bd = 0 is SSKIP_ERR_INVALID_ARG.
+ */
+int sskip_attn_step(const void* q, const void* k, const void* v, void* o, float* lse, int Bp,
+                    int L, int causal, int Br, int Bc, unsigned long long* prefill_count,
+                    const void* dq, const void* kcache, const void* vcache, const int* seqlens,
+                    void* dout, float* dlse, int Bd, int Lmax, int num_splits, void* workspace,
+                    size_t workspace_bytes, unsigned long long* decode_count, int Hq, int Hkv,
+                    int d, float sm_scale, float tsf_prefill, float tsf_decode, void* stream);
+
+/*
  * Token reordering along a 3-D Hilbert curve (SpargeAttn article, "Hilbert
  * 曲线置换": the T x H x W visual tokens are laid out along a Hilbert curve
  * before attention so that the tokens of one tile form a compact 3-D region,

@@ -134,3 +134,24 @@ def unit_slice_margins(x, w, b, hq, i, R, tsf):
                 out[s, j] = mg[a:e].min()
         prefix = np.maximum(prefix, ml)
     return out
+
+
+def compare_prefill_units(w, x, g, ora, units):
+    """Compare GPU prefill outputs (full layout: g["o"] [B,Hq,L,d],
+    g["lse"], g["tile_state"]) with per-unit oracle outputs for (b, hq, i)
+    units (ora["o"] [n,Br,d], ora["lse"], ora["tile_state"], ora["tile_margin"]).
+    A unit whose decisions flipped at a near-tie is checked against fp64
+    attention restricted to the GPU's own kept tiles. Returns the flip count."""
+    flips = 0
+    for n, (b, hq, i) in enumerate(units):
+        r0, r1 = i * w.Br, min(w.L, (i + 1) * w.Br)
+        st_g = g["tile_state"][b, hq, i]
+        diff = check_tiles(st_g, ora["tile_state"][n], ora["tile_margin"][n])
+        if diff.any():
+            flips += int(diff.sum())
+            o_ref, lse_ref = unit_restricted_reference(x, w, b, hq, i, np.nonzero(st_g == 1)[0])
+        else:
+            o_ref, lse_ref = ora["o"][n, :r1 - r0], ora["lse"][n, :r1 - r0]
+        check_rows(g["o"][b, hq, r0:r1], g["lse"][b, hq, r0:r1], o_ref, lse_ref,
+                   what=f"unit {(b, hq, i)}")
+    return flips

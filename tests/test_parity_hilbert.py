@@ -9,8 +9,7 @@ import block_sparse_long_tiled_b200 as sk
 import oracle
 import synth
 from oracle.hilbert import hilbert_order
-from parity_helpers import (bf16_host, check_counts, check_rows, check_tiles, to_device,
-                            unit_restricted_reference)
+from parity_helpers import bf16_host, check_counts, compare_prefill_units, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -57,7 +56,10 @@ def test_permute_rows_flags_a_bad_index():
 
 def small_video(**kw):
     base = dict(synth.VIDEO_DIT_PREFILL.__dict__)
-    base.update(name="t", B=1, Hq=2, Hkv=2, L=350, video_grid=(5, 8, 9))
+    # A 5 x 16 x 25 grid: enough keys per row that |O| stays below ~1.8, as
+    # on the full workload (a smaller grid gives peaked rows with |O| ~ 3,
+    # where bf16 rounding of O alone nears the 1e-2 bound); t = 1000 / 2000.
+    base.update(name="t", B=1, Hq=2, Hkv=2, L=2000, video_grid=(5, 16, 25), tsf=1000.0)
     base.update(kw)
     return synth.PrefillWorkload(**base)
 
@@ -66,7 +68,7 @@ def reordered_parity(w, x, perm, n_units=None, seed=0):
     dev_perm = torch.from_numpy(perm).cuda()
     q, k, v = to_device(x["q"]), to_device(x["k"]), to_device(x["v"])
     out = sk.prefill_reordered(q, k, v, dev_perm, sm_scale=w.scale,
-                               threshold_scale_factor=w.tsf, Br=w.Br, Bc=w.Bc)
+                               threshold_scale_factor=w.tsf, Br=w.Br, Bc=w.Bc, with_tiles=True)
     torch.cuda.synchronize()
     assert sk.sskip_get_status() == sk.SSKIP_OK
     xp = {n: np.ascontiguousarray(x[n][:, :, perm]) for n in ("q", "k", "v")}
@@ -78,12 +80,10 @@ def reordered_parity(w, x, perm, n_units=None, seed=0):
                  for i in np.linspace(0, w.n_q - 1, n_units).astype(int)]
     ora = oracle.prefill(xp["q"], xp["k"], xp["v"], causal=False, sm_scale=w.scale, tsf=w.tsf,
                          Br=w.Br, Bc=w.Bc, units=np.array(units, np.int32), want_margin=True)
-    o = bf16_host(out["o"])[:, :, perm]          # back into the reordered frame
-    lse = out["lse"].cpu().numpy()[:, :, perm]
-    for n, (b, h, i) in enumerate(units):
-        r0, r1 = i * w.Br, min(w.L, (i + 1) * w.Br)
-        o_ref, lse_ref = ora["o"][n, :r1 - r0], ora["lse"][n, :r1 - r0]
-        check_rows(o[b, h, r0:r1], lse[b, h, r0:r1], o_ref, lse_ref, what=f"unit {(b, h, i)}")
+    # Outputs came back in the original order; compare in the reordered frame.
+    g = {"o": bf16_host(out["o"])[:, :, perm], "lse": out["lse"].cpu().numpy()[:, :, perm],
+         "tile_state": out["tile_state"].cpu().numpy()}
+    compare_prefill_units(w, xp, g, ora, units)
     return out
 
 
