@@ -22,7 +22,8 @@ def _built():
 
 def make_case():
     pw = PrefillWorkload(name="p", B=1, Hq=8, Hkv=2, L=1000, d=128, causal=True, Br=128, Bc=128,
-                         tsf=0.0, seed=61)
+                         tsf=0.0, seed=61, q_shift=0.5, hot_frac=0.15, hot_gain=2.0,
+                         sink_keys=4, sink_gain=3.0)
     dw = DecodeWorkload(name="d", B=4, Hq=8, Hkv=2, d=128, Lmin=900, Lmax=3000, Bc=64,
                         num_splits=4, tsf=0.0, seed=62)
     px = synth.prefill_inputs(pw, "rms")
