@@ -295,7 +295,7 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
                                       Br=w.Br, Bc=w.Bc, skip_count=t["cnt"], tile_state=tiles,
                                       stream=stream)
             legs.append({"name": f"prefill_{rd}", "kind": "prefill", "reading": rd, "t": t,
-                         "host": x, "run": run, "launches": 1})
+                         "host": x, "run": run, "launches": 1, "w": w})
             if rd in warp_readings:
                 # Same inputs, vote taken per 32-row warp slice.
                 tw = dict(t, o=torch.empty_like(t["q"]),
@@ -398,7 +398,8 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
 
     # ---- end to end through the public API: pinned host in, host out
     ems, io_bytes = ({}, (0, 0)) if args.no_e2e else time_e2e(legs, flush, stream, new_events,
-                                                             timed, args.steps)
+                                                             timed, args.steps,
+                                                             args.e2e_kv_per_chunk)
 
     if rank == 0:
         print(json.dumps(report(args, w, dw, world, legs, ms, ms_dense, ems, io_bytes, peaks,
@@ -408,7 +409,7 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
         dist.destroy_process_group()
 
 
-def time_e2e(legs, flush, stream, new_events, timed, steps):
+def time_e2e(legs, flush, stream, new_events, timed, steps, kv_per_chunk=0):
     """Same steps with each leg's inputs copied host->device from pinned memory
     and its outputs copied back inside the timed region."""
     import torch
@@ -430,16 +431,28 @@ def time_e2e(legs, flush, stream, new_events, timed, steps):
         h2d += sum(int(v.numel() * v.element_size()) for v in leg["pin_in"].values())
         d2h += sum(int(v.numel() * v.element_size()) for v in leg["pin_out"])
 
+    import block_sparse_long_tiled_b200 as sk
+
     def e2e_step(ev):
         for leg in legs:
             t = leg["t"]
             flush.zero_()
             ev[leg["name"]][0].record(stream)
-            for n, hv in leg["pin_in"].items():
-                leg["dev_in"][n].copy_(hv, non_blocking=True)
-            leg["run"]()
-            leg["pin_out"][0].copy_(t["o"], non_blocking=True)
-            leg["pin_out"][1].copy_(t["lse"], non_blocking=True)
+            if leg["kind"] == "prefill":
+                # Host buffers through the library's overlapped host-memory call.
+                w = leg["w"]
+                host = dict(leg["pin_in"], o=leg["pin_out"][0], lse=leg["pin_out"][1])
+                dev = dict(leg["dev_in"], o=t["o"], lse=t["lse"])
+                sk.sskip_attn_prefill_host(host, dev, causal=w.causal, sm_scale=w.scale,
+                                           threshold_scale_factor=w.tsf, Br=w.Br, Bc=w.Bc,
+                                           kv_per_chunk=kv_per_chunk, skip_count=t["cnt"],
+                                           stream=stream)
+            else:
+                for n, hv in leg["pin_in"].items():
+                    leg["dev_in"][n].copy_(hv, non_blocking=True)
+                leg["run"]()
+                leg["pin_out"][0].copy_(t["o"], non_blocking=True)
+                leg["pin_out"][1].copy_(t["lse"], non_blocking=True)
             ev[leg["name"]][1].record(stream)
 
     return timed(e2e_step, steps, only=[leg["name"] for leg in legs]), (h2d, d2h)
@@ -869,6 +882,8 @@ def main(argv=None):
     ap.add_argument("--cpu-heads", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-kv-per-chunk", type=int, default=0,
+                    help="kv heads per copy/compute group of the host-memory prefill (0: auto)")
     ap.add_argument("--no-control", action="store_true",
                     help="skip the tsf = 0 (skipping disabled) control timing")
     ap.add_argument("--decode-readings", choices=["all", "headline"], default="all")

@@ -28,7 +28,7 @@ EXPORTS = ("sskip_version", "sskip_status_string", "sskip_device_supported",
            "sskip_attn_decode_workspace_size",
            "sskip_attn_decode", "sskip_attn_decode_ex", "sskip_attn_decode_crit",
            "sskip_attn_decode_noalloc", "sskip_calibrate_factor", "sskip_hilbert3d_order",
-           "sskip_permute_rows", "sskip_attn_step",
+           "sskip_permute_rows", "sskip_attn_step", "sskip_attn_prefill_host",
            "sskip_get_status", "sskip_selftest_watchdog")
 
 # Size of the library's fixed decode scratch (see sskip_attn_decode_noalloc).
@@ -82,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.sskip_hilbert3d_order.argtypes = [I, I, I, I, P]
         L.sskip_permute_rows.restype = I
         L.sskip_permute_rows.argtypes = [P, P, P, ctypes.c_longlong, I, I, I, P]
+        L.sskip_attn_prefill_host.restype = I
+        L.sskip_attn_prefill_host.argtypes = [P] * 10 + [I, I, I, I, I, I, F, F, I, I, I, P, P]
         L.sskip_attn_step.restype = I
         L.sskip_attn_step.argtypes = ([P, P, P, P, P, I, I, I, I, I, P] +
                                       [P, P, P, P, P, P, I, I, I, P, Z, P] +
@@ -158,6 +160,25 @@ def sskip_attn_prefill_vote(q, k, v, o, lse, *, causal: bool, sm_scale: float,
                                        int(vote_rows), _ptr(counts), _ptr(tile_state),
                                        _ptr(slice_mask), _ptr(tile_crit), _stream(stream))
     _check(rc, "sskip_attn_prefill_vote")
+
+
+def sskip_attn_prefill_host(host: dict, dev: dict, *, causal: bool, sm_scale: float,
+                            threshold_scale_factor: float, Br: int = 128, Bc: int = 128,
+                            kv_per_chunk: int = 0, skip_count=None, stream=None) -> None:
+    """Marshal host tensors (q, k, v, o, lse; pinned for overlap) and device
+    staging tensors of the same shapes into sskip_attn_prefill_host."""
+    for t in (host["q"], host["k"], host["v"], host["o"], dev["q"], dev["k"], dev["v"], dev["o"]):
+        _bf16_view(t)
+    if host["q"].is_cuda or not dev["q"].is_cuda:
+        raise ValueError("host tensors on the CPU, staging tensors on the GPU")
+    B, Hq, L, d = host["q"].shape
+    Hkv = host["k"].shape[1]
+    rc = lib().sskip_attn_prefill_host(*(_ptr(host[n]) for n in ("q", "k", "v", "o", "lse")),
+                                       *(_ptr(dev[n]) for n in ("q", "k", "v", "o", "lse")),
+                                       B, Hq, Hkv, L, d, int(bool(causal)), float(sm_scale),
+                                       float(threshold_scale_factor), int(Br), int(Bc),
+                                       int(kv_per_chunk), _ptr(skip_count), _stream(stream))
+    _check(rc, "sskip_attn_prefill_host")
 
 
 def sskip_attn_decode_workspace_size(B: int, Hq: int, d: int, num_splits: int) -> int:

@@ -156,7 +156,8 @@ namespace {
 int prefill_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                  int Hkv, int L, int d, int causal, float sm_scale, float threshold_scale_factor,
                  int Br, int Bc, int vote_rows, unsigned long long* counts, int n_counts,
-                 uint8_t* tile_state, uint8_t* slice_mask, float* tile_crit, void* stream) {
+                 uint8_t* tile_state, uint8_t* slice_mask, float* tile_crit, void* stream,
+                 bool zero_counts = true) {
   if (!q || !k || !v || !o || !lse) return SSKIP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(counts) & 7u) ||
@@ -199,7 +200,7 @@ int prefill_impl(const void* q, const void* k, const void* v, void* o, float* ls
   p.log2_t = p.t_positive ? (float)std::log2((double)threshold_scale_factor / (double)L)
                           : -INFINITY;
 
-  if (counts &&
+  if (counts && zero_counts &&
       cudaMemsetAsync(counts, 0, (size_t)n_counts * sizeof(unsigned long long), st) != cudaSuccess)
     return SSKIP_ERR_CUDA;
   if (tile_state &&
@@ -598,4 +599,118 @@ SSKIP_API int sskip_attn_step(const void* q, const void* k, const void* v, void*
                                 sm_scale, tsf_decode, kDecBc, num_splits, workspace,
                                 workspace_bytes, decode_count, nullptr, stream);
   return SSKIP_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Prefill from and to host memory, with the copies overlapped with the
+// kernels: the work is cut into groups of kv heads (each group's query heads,
+// keys, values, outputs and lse rows are contiguous in the [B, H, L, ...]
+// layouts), and group i's copy in, group i-1's prefill and group i-2's copy
+// out run at the same time on three streams.
+namespace sskip {
+namespace {
+
+struct CopyStreams {
+  cudaStream_t in = nullptr, out = nullptr;
+};
+
+// Two non-blocking copy streams per device, created on first use and kept
+// for the life of the process.
+int copy_streams(CopyStreams* cs) {
+  static std::mutex mu;
+  static CopyStreams per_dev[64];
+  const int dev = current_device();
+  if (dev < 0 || dev >= 64) return SSKIP_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  CopyStreams& c = per_dev[dev];
+  if (!c.in && cudaStreamCreateWithFlags(&c.in, cudaStreamNonBlocking) != cudaSuccess)
+    return SSKIP_ERR_CUDA;
+  if (!c.out && cudaStreamCreateWithFlags(&c.out, cudaStreamNonBlocking) != cudaSuccess)
+    return SSKIP_ERR_CUDA;
+  *cs = c;
+  return SSKIP_OK;
+}
+
+}  // namespace
+}  // namespace sskip
+
+SSKIP_API int sskip_attn_prefill_host(const void* q_h, const void* k_h, const void* v_h, void* o_h,
+                                      float* lse_h, void* q_d, void* k_d, void* v_d, void* o_d,
+                                      float* lse_d, int B, int Hq, int Hkv, int L, int d,
+                                      int causal, float sm_scale, float threshold_scale_factor,
+                                      int Br, int Bc, int kv_per_chunk,
+                                      unsigned long long* skip_count, void* stream) {
+  if (!q_h || !k_h || !v_h || !o_h || !lse_h || !q_d || !k_d || !v_d || !o_d || !lse_d)
+    return SSKIP_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0 || kv_per_chunk < 0)
+    return SSKIP_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SSKIP_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  const int n_units = (L + kPfUnitRows - 1) / kPfUnitRows;
+  int kc = kv_per_chunk;
+  if (kc == 0) {  // at least two waves of CTAs per group on a 148-SM part
+    const int per_kv = G * n_units;
+    kc = std::max(1, (296 + per_kv - 1) / per_kv);
+  }
+  kc = std::min(kc, Hkv);
+  CopyStreams cs;
+  int rc = copy_streams(&cs);
+  if (rc != SSKIP_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t row = (size_t)L * d * 2;  // bytes of one head's [L, d] bf16 matrix
+  const int n_groups = (Hkv + kc - 1) / kc;
+  const int n_chunks = B * n_groups;
+  // ev[2c]: chunk c copied in; ev[2c + 1]: chunk c computed; then start, end.
+  std::vector<cudaEvent_t> ev(2 * n_chunks + 2, nullptr);
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      rc = SSKIP_ERR_CUDA;
+      break;
+    }
+  if (rc == SSKIP_OK && skip_count &&
+      cudaMemsetAsync(skip_count, 0, 2 * sizeof(unsigned long long), st) != cudaSuccess)
+    rc = SSKIP_ERR_CUDA;
+  // Copies start only after the work already queued on the caller's stream.
+  if (rc == SSKIP_OK && (cudaEventRecord(ev[2 * n_chunks], st) != cudaSuccess ||
+                         cudaStreamWaitEvent(cs.in, ev[2 * n_chunks], 0) != cudaSuccess ||
+                         cudaStreamWaitEvent(cs.out, ev[2 * n_chunks], 0) != cudaSuccess))
+    rc = SSKIP_ERR_CUDA;
+  auto h2d = [&](void* dst, const void* src, size_t off, size_t n) {
+    return cudaMemcpyAsync(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off, n,
+                           cudaMemcpyHostToDevice, cs.in) == cudaSuccess;
+  };
+  auto d2h = [&](void* dst, const void* src, size_t off, size_t n) {
+    return cudaMemcpyAsync(static_cast<char*>(dst) + off, static_cast<const char*>(src) + off, n,
+                           cudaMemcpyDeviceToHost, cs.out) == cudaSuccess;
+  };
+  for (int c = 0; rc == SSKIP_OK && c < n_chunks; ++c) {
+    const int b = c / n_groups, kv0 = (c % n_groups) * kc, nk = std::min(kc, Hkv - kv0);
+    const size_t qo = ((size_t)b * Hq + (size_t)kv0 * G) * row, qn = (size_t)nk * G * row;
+    const size_t ko = ((size_t)b * Hkv + kv0) * row, kn = (size_t)nk * row;
+    const size_t lo = ((size_t)b * Hq + (size_t)kv0 * G) * L * 4, ln = (size_t)nk * G * L * 4;
+    if (!h2d(q_d, q_h, qo, qn) || !h2d(k_d, k_h, ko, kn) || !h2d(v_d, v_h, ko, kn) ||
+        cudaEventRecord(ev[2 * c], cs.in) != cudaSuccess ||
+        cudaStreamWaitEvent(st, ev[2 * c], 0) != cudaSuccess) {
+      rc = SSKIP_ERR_CUDA;
+      break;
+    }
+    rc = prefill_impl(static_cast<const char*>(q_d) + qo, static_cast<const char*>(k_d) + ko,
+                      static_cast<const char*>(v_d) + ko, static_cast<char*>(o_d) + qo,
+                      reinterpret_cast<float*>(reinterpret_cast<char*>(lse_d) + lo), 1, nk * G, nk,
+                      L, d, causal, sm_scale, threshold_scale_factor, Br, Bc, Br, skip_count, 2,
+                      nullptr, nullptr, nullptr, stream, /*zero_counts=*/false);
+    if (rc != SSKIP_OK) break;
+    if (cudaEventRecord(ev[2 * c + 1], st) != cudaSuccess ||
+        cudaStreamWaitEvent(cs.out, ev[2 * c + 1], 0) != cudaSuccess ||
+        !d2h(o_h, o_d, qo, qn) ||
+        !d2h(lse_h, lse_d, lo, ln))
+      rc = SSKIP_ERR_CUDA;
+  }
+  // The caller's stream completes only after the last copy out.
+  if (rc == SSKIP_OK && (cudaEventRecord(ev[2 * n_chunks + 1], cs.out) != cudaSuccess ||
+                         cudaStreamWaitEvent(st, ev[2 * n_chunks + 1], 0) != cudaSuccess))
+    rc = SSKIP_ERR_CUDA;
+  for (auto& e : ev)
+    if (e) cudaEventDestroy(e);  // released once the recorded work completes
+  return rc;
 }

@@ -137,6 +137,33 @@ int sskip_attn_prefill_vote(const void* q, const void* k, const void* v, void* o
                             uint8_t* slice_mask, float* tile_crit, void* stream);
 
 /*
+ * Prefill from HOST memory to HOST memory, the copies overlapped with the
+ * kernels.  Computes exactly sskip_attn_prefill_ex (no tile record) on the
+ * same arguments: q_h, k_h, v_h, o_h, lse_h are host buffers in the layouts
+ * above (pinned memory lets the copies overlap; pageable memory works but
+ * serialises them); q_d, k_d, v_d, o_d, lse_d are device buffers of the same
+ * sizes, owned by the caller (inputs are staged there; their contents after
+ * the call are the staged inputs and the outputs).
+ *
+ * The kv heads of each batch entry are cut into groups of kv_per_chunk (0 =
+ * pick so that a group fills at least two waves of CTAs on a 148-SM part);
+ * a group's query heads, keys, values, outputs and lse rows are contiguous,
+ * and group c's host-to-device copy, group c-1's prefill and group c-2's
+ * device-to-host copy run concurrently on two library-owned copy streams and
+ * `stream`.  Every query tile is computed by the same kernel code as in the
+ * one-shot call, so the outputs are bit-identical to it.
+ * skip_count: optional device uint64[2], summed over the groups.
+ * The call returns after enqueueing; the outputs are in host memory once
+ * `stream` has completed (it waits for the last copy).  The two copy streams
+ * are created on first use, once per device, and kept for the process's life.
+ */
+int sskip_attn_prefill_host(const void* q_h, const void* k_h, const void* v_h, void* o_h,
+                            float* lse_h, void* q_d, void* k_d, void* v_d, void* o_d, float* lse_d,
+                            int B, int Hq, int Hkv, int L, int d, int causal, float sm_scale,
+                            float threshold_scale_factor, int Br, int Bc, int kv_per_chunk,
+                            unsigned long long* skip_count, void* stream);
+
+/*
  * Decode: one new query token per sequence against a contiguous KV cache,
  * split over the key axis and merged by log-sum-exp (the bandwidth-bound
  * phase of the article's "Skip Softmax 带来了哪些实战好处" section: a skipped

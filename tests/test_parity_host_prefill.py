@@ -1,0 +1,80 @@
+"""GPU checks of the host-buffer prefill (sskip_attn_prefill_host): for every
+way of cutting the kv heads into groups, pinned or pageable host memory, its
+outputs and skip counts are bit-identical to the one-shot device call, which
+the other parity tests compare with the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_long_tiled_b200 as sk
+import synth
+from parity_helpers import to_device
+from synth import PrefillWorkload
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from block_sparse_long_tiled_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+
+
+def host_bf16(bits, pin):
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.pin_memory() if pin else t.clone()
+
+
+@pytest.mark.parametrize("kv_per_chunk", [0, 1, 3, 8])
+@pytest.mark.parametrize("pin", [True, False])
+@pytest.mark.parametrize("w", [
+    PrefillWorkload(name="h", B=2, Hq=8, Hkv=4, L=700, d=128, causal=True, Br=128, Bc=128,
+                    tsf=60.0, seed=71, q_shift=0.5, hot_frac=0.15, hot_gain=2.0, sink_keys=4,
+                    sink_gain=3.0),
+    PrefillWorkload(name="h", B=1, Hq=6, Hkv=3, L=333, d=64, causal=False, Br=64, Bc=64,
+                    tsf=30.0, seed=72, q_shift=0.5, hot_frac=0.15, hot_gain=2.0, sink_keys=4,
+                    sink_gain=3.0),
+], ids=["gqa_causal_d128", "noncausal_d64_br64"])
+def test_host_prefill_equals_device_call(w, pin, kv_per_chunk):
+    x = synth.prefill_inputs(w, "rms")
+    q, k, v = to_device(x["q"]), to_device(x["k"]), to_device(x["v"])
+    ref = sk.prefill(q, k, v, causal=w.causal, sm_scale=w.scale, threshold_scale_factor=w.tsf,
+                     Br=w.Br, Bc=w.Bc)
+    host = {n: host_bf16(x[n], pin) for n in ("q", "k", "v")}
+    host["o"] = torch.empty_like(host["q"])
+    host["lse"] = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32)
+    if pin:
+        host["o"], host["lse"] = host["o"].pin_memory(), host["lse"].pin_memory()
+    dev = {n: torch.empty_like(t, device="cuda") for n, t in host.items()}
+    cnt = torch.zeros(2, dtype=torch.int64, device="cuda")
+    sk.sskip_attn_prefill_host(host, dev, causal=w.causal, sm_scale=w.scale,
+                               threshold_scale_factor=w.tsf, Br=w.Br, Bc=w.Bc,
+                               kv_per_chunk=kv_per_chunk, skip_count=cnt)
+    torch.cuda.current_stream().synchronize()
+    assert sk.sskip_get_status() == sk.SSKIP_OK
+    assert torch.equal(host["o"], ref["o"].cpu())
+    assert torch.equal(host["lse"], ref["lse"].cpu())
+    assert cnt.cpu().tolist() == ref["counts"].cpu().tolist()
+    assert ref["counts"].cpu().tolist()[0] > 0
+
+
+def test_host_prefill_twice_in_a_row_reuses_the_staging_buffers():
+    w = PrefillWorkload(name="h", B=1, Hq=4, Hkv=2, L=512, d=128, causal=True, Br=128, Bc=128,
+                        tsf=60.0, seed=73)
+    outs = []
+    for seed in (73, 74):
+        x = synth.prefill_inputs(w.replace(seed=seed), "rms")
+        host = {n: host_bf16(x[n], True) for n in ("q", "k", "v")}
+        host["o"] = torch.empty_like(host["q"]).pin_memory()
+        host["lse"] = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32).pin_memory()
+        if not outs:
+            dev = {n: torch.empty_like(t, device="cuda") for n, t in host.items()}
+        sk.sskip_attn_prefill_host(host, dev, causal=True, sm_scale=w.scale,
+                                   threshold_scale_factor=w.tsf, kv_per_chunk=1)
+        ref = sk.prefill(to_device(x["q"]), to_device(x["k"]), to_device(x["v"]), causal=True,
+                         sm_scale=w.scale, threshold_scale_factor=w.tsf)
+        torch.cuda.synchronize()
+        assert torch.equal(host["o"], ref["o"].cpu())
+        outs.append(host["o"])
+    assert not torch.equal(outs[0], outs[1])
