@@ -648,9 +648,9 @@ SSKIP_API int sskip_attn_prefill_host(const void* q_h, const void* k_h, const vo
   const int G = Hq / Hkv;
   const int n_units = (L + kPfUnitRows - 1) / kPfUnitRows;
   int kc = kv_per_chunk;
-  if (kc == 0) {  // at least two waves of CTAs per group on a 148-SM part
+  if (kc == 0) {  // the smallest group that still fills one wave of a 148-SM part
     const int per_kv = G * n_units;
-    kc = std::max(1, (296 + per_kv - 1) / per_kv);
+    kc = std::max(1, (148 + per_kv - 1) / per_kv);
   }
   kc = std::min(kc, Hkv);
   CopyStreams cs;

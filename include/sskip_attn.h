@@ -29,7 +29,10 @@
  *    by the caller, 16-byte aligned, densely packed in the layouts stated.
  *    bf16 tensors are raw IEEE bfloat16 (uint16 storage).
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
- *    Every call is asynchronous on that stream and allocates nothing.
+ *    Every device call is asynchronous on that stream and allocates no device
+ *    memory.  sskip_attn_prefill_host also creates two copy streams once per
+ *    device and a few events per call.  sskip_calibrate_factor and
+ *    sskip_hilbert3d_order are host-only and synchronous.
  *  - The return value reports argument validation and launch errors
  *    synchronously (sskip_status).  Errors found on the device while a kernel
  *    runs (a bounded wait that ran out) are latched in a per-device status
@@ -146,7 +149,8 @@ int sskip_attn_prefill_vote(const void* q, const void* k, const void* v, void* o
  * the call are the staged inputs and the outputs).
  *
  * The kv heads of each batch entry are cut into groups of kv_per_chunk (0 =
- * pick so that a group fills at least two waves of CTAs on a 148-SM part);
+ * the smallest group that fills one wave of CTAs on a 148-SM part: small
+ * groups shorten the pipeline's fill and drain);
  * a group's query heads, keys, values, outputs and lse rows are contiguous,
  * and group c's host-to-device copy, group c-1's prefill and group c-2's
  * device-to-host copy run concurrently on two library-owned copy streams and
