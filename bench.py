@@ -331,7 +331,7 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
                                      skip_count=t["cnt"], tile_state=tiles, stream=stream)
             legs.append({"name": f"decode_{rd}", "kind": "decode", "reading": rd, "t": t,
                          "host": {"q": dx["q"], "seqlens": dx["seqlens"]}, "run": run,
-                         "launches": 2})
+                         "launches": 2, "dw": dw})
             del dx
 
     # ---- one untimed pass with tile records: skip counts, FLOPs, bytes moved
@@ -448,11 +448,14 @@ def time_e2e(legs, flush, stream, new_events, timed, steps, kv_per_chunk=0):
                                            kv_per_chunk=kv_per_chunk, skip_count=t["cnt"],
                                            stream=stream)
             else:
-                for n, hv in leg["pin_in"].items():
-                    leg["dev_in"][n].copy_(hv, non_blocking=True)
-                leg["run"]()
-                leg["pin_out"][0].copy_(t["o"], non_blocking=True)
-                leg["pin_out"][1].copy_(t["lse"], non_blocking=True)
+                dw = leg["dw"]
+                host = {"q": leg["pin_in"]["q"], "seqlens": leg["pin_in"]["lens"],
+                        "o": leg["pin_out"][0], "lse": leg["pin_out"][1]}
+                dev = {"q": t["q"], "seqlens": t["lens"], "o": t["o"], "lse": t["lse"]}
+                sk.sskip_attn_decode_host(host, dev, t["kc"], t["vc"], sm_scale=dw.scale,
+                                          threshold_scale_factor=dw.tsf, Bc=dw.Bc,
+                                          num_splits=dw.num_splits, workspace=t["ws"],
+                                          skip_count=t["cnt"], stream=stream)
             ev[leg["name"]][1].record(stream)
 
     return timed(e2e_step, steps, only=[leg["name"] for leg in legs]), (h2d, d2h)

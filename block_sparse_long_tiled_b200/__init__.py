@@ -29,6 +29,7 @@ EXPORTS = ("sskip_version", "sskip_status_string", "sskip_device_supported",
            "sskip_attn_decode", "sskip_attn_decode_ex", "sskip_attn_decode_crit",
            "sskip_attn_decode_noalloc", "sskip_calibrate_factor", "sskip_hilbert3d_order",
            "sskip_permute_rows", "sskip_attn_step", "sskip_attn_prefill_host",
+           "sskip_attn_decode_host",
            "sskip_get_status", "sskip_selftest_watchdog")
 
 # Size of the library's fixed decode scratch (see sskip_attn_decode_noalloc).
@@ -84,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.sskip_permute_rows.argtypes = [P, P, P, ctypes.c_longlong, I, I, I, P]
         L.sskip_attn_prefill_host.restype = I
         L.sskip_attn_prefill_host.argtypes = [P] * 10 + [I, I, I, I, I, I, F, F, I, I, I, P, P]
+        L.sskip_attn_decode_host.restype = I
+        L.sskip_attn_decode_host.argtypes = [P] * 10 + [I, I, I, I, I, F, F, I, I, P, Z, P, P]
         L.sskip_attn_step.restype = I
         L.sskip_attn_step.argtypes = ([P, P, P, P, P, I, I, I, I, I, P] +
                                       [P, P, P, P, P, P, I, I, I, P, Z, P] +
@@ -179,6 +182,25 @@ def sskip_attn_prefill_host(host: dict, dev: dict, *, causal: bool, sm_scale: fl
                                        float(threshold_scale_factor), int(Br), int(Bc),
                                        int(kv_per_chunk), _ptr(skip_count), _stream(stream))
     _check(rc, "sskip_attn_prefill_host")
+
+
+def sskip_attn_decode_host(host: dict, dev: dict, kcache, vcache, *, sm_scale: float,
+                           threshold_scale_factor: float, Bc: int = 64, num_splits: int = 16,
+                           workspace=None, skip_count=None, stream=None) -> None:
+    """Marshal host q, seqlens, o, lse (pinned for async copies), their device
+    staging buffers and the device-resident caches into sskip_attn_decode_host."""
+    for t in (host["q"], host["o"], dev["q"], dev["o"], kcache, vcache):
+        _bf16_view(t)
+    B, Hq, d = host["q"].shape
+    Hkv, Lmax = kcache.shape[1], kcache.shape[2]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().sskip_attn_decode_host(*(_ptr(host[n]) for n in ("q", "seqlens", "o", "lse")),
+                                      *(_ptr(dev[n]) for n in ("q", "seqlens", "o", "lse")),
+                                      _ptr(kcache), _ptr(vcache), B, Hq, Hkv, Lmax, d,
+                                      float(sm_scale), float(threshold_scale_factor), int(Bc),
+                                      int(num_splits), _ptr(workspace), ws_bytes,
+                                      _ptr(skip_count), _stream(stream))
+    _check(rc, "sskip_attn_decode_host")
 
 
 def sskip_attn_decode_workspace_size(B: int, Hq: int, d: int, num_splits: int) -> int:

@@ -714,3 +714,29 @@ SSKIP_API int sskip_attn_prefill_host(const void* q_h, const void* k_h, const vo
     if (e) cudaEventDestroy(e);  // released once the recorded work completes
   return rc;
 }
+
+SSKIP_API int sskip_attn_decode_host(const void* q_h, const int* seqlens_h, void* o_h, float* lse_h,
+                                     void* q_d, int* seqlens_d, void* o_d, float* lse_d,
+                                     const void* kcache, const void* vcache, int B, int Hq,
+                                     int Hkv, int Lmax, int d, float sm_scale,
+                                     float threshold_scale_factor, int Bc, int num_splits,
+                                     void* workspace, size_t workspace_bytes,
+                                     unsigned long long* skip_count, void* stream) {
+  if (!q_h || !seqlens_h || !o_h || !lse_h || !q_d || !seqlens_d || !o_d || !lse_d)
+    return SSKIP_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || (d != 64 && d != 128)) return SSKIP_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t qn = (size_t)B * Hq * d * 2, ln = (size_t)B * Hq * 4;
+  if (cudaMemcpyAsync(q_d, q_h, qn, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(seqlens_d, seqlens_h, (size_t)B * 4, cudaMemcpyHostToDevice, st) !=
+          cudaSuccess)
+    return SSKIP_ERR_CUDA;
+  const int rc = sskip_attn_decode_ex(q_d, kcache, vcache, seqlens_d, o_d, lse_d, B, Hq, Hkv,
+                                      Lmax, d, sm_scale, threshold_scale_factor, Bc, num_splits,
+                                      workspace, workspace_bytes, skip_count, nullptr, stream);
+  if (rc != SSKIP_OK) return rc;
+  if (cudaMemcpyAsync(o_h, o_d, qn, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(lse_h, lse_d, ln, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return SSKIP_ERR_CUDA;
+  return SSKIP_OK;
+}

@@ -289,6 +289,23 @@ int sskip_attn_decode_noalloc(const void* q, const void* kcache, const void* vca
                               unsigned long long* skip_count, void* stream);
 
 /*
+ * Decode with the per-step tensors in HOST memory: q_h [B, Hq, d] bf16 and
+ * seqlens_h [B] int32 are copied to the caller's device buffers q_d and
+ * seqlens_d, the decode runs exactly as sskip_attn_decode_ex (no tile record)
+ * against the device-resident kcache / vcache, and o_d / lse_d are copied
+ * back to o_h [B, Hq, d] bf16 and lse_h [B, Hq] fp32, all in order on
+ * `stream` (the step's copies are a few hundred KB: nothing to overlap).
+ * Pinned host memory keeps the copies asynchronous.  Validation as in
+ * sskip_attn_decode_ex.
+ */
+int sskip_attn_decode_host(const void* q_h, const int* seqlens_h, void* o_h, float* lse_h,
+                           void* q_d, int* seqlens_d, void* o_d, float* lse_d,
+                           const void* kcache, const void* vcache, int B, int Hq, int Hkv,
+                           int Lmax, int d, float sm_scale, float threshold_scale_factor, int Bc,
+                           int num_splits, void* workspace, size_t workspace_bytes,
+                           unsigned long long* skip_count, void* stream);
+
+/*
  * One serving step of one attention layer with a factor per phase: the
  * TensorRT-LLM article ("实战演练") lets threshold_scale_factor be a single
  * number or a {prefill: 1000, decode: 500} pair, each divided by its own

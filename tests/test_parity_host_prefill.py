@@ -78,3 +78,31 @@ def test_host_prefill_twice_in_a_row_reuses_the_staging_buffers():
         assert torch.equal(host["o"], ref["o"].cpu())
         outs.append(host["o"])
     assert not torch.equal(outs[0], outs[1])
+
+
+@pytest.mark.parametrize("pin", [True, False])
+def test_host_decode_equals_device_call(pin):
+    from synth import DecodeWorkload
+    w = DecodeWorkload(name="hd", B=5, Hq=8, Hkv=2, d=128, Lmin=200, Lmax=1500, Bc=64,
+                       num_splits=4, tsf=40.0, seed=75)
+    x = synth.decode_inputs(w, "rms")
+    kc, vc = to_device(x["kcache"]), to_device(x["vcache"])
+    lens = torch.from_numpy(x["seqlens"]).cuda()
+    q = to_device(x["q"])
+    ref = sk.decode(q, kc, vc, lens, sm_scale=w.scale, threshold_scale_factor=w.tsf, Bc=w.Bc,
+                    num_splits=w.num_splits)
+    host = {"q": host_bf16(x["q"], pin), "seqlens": torch.from_numpy(x["seqlens"]).clone(),
+            "o": torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16),
+            "lse": torch.empty((w.B, w.Hq), dtype=torch.float32)}
+    if pin:
+        host = {n: t.pin_memory() for n, t in host.items()}
+    dev = {n: torch.empty_like(t, device="cuda") for n, t in host.items()}
+    ws = torch.empty(sk.sskip_attn_decode_workspace_size(w.B, w.Hq, w.d, w.num_splits),
+                     dtype=torch.uint8, device="cuda")
+    cnt = torch.zeros(2, dtype=torch.int64, device="cuda")
+    sk.sskip_attn_decode_host(host, dev, kc, vc, sm_scale=w.scale, threshold_scale_factor=w.tsf,
+                              Bc=w.Bc, num_splits=w.num_splits, workspace=ws, skip_count=cnt)
+    torch.cuda.current_stream().synchronize()
+    assert sk.sskip_get_status() == sk.SSKIP_OK
+    assert torch.equal(host["o"], ref["o"].cpu()) and torch.equal(host["lse"], ref["lse"].cpu())
+    assert cnt.cpu().tolist() == ref["counts"].cpu().tolist() and cnt.cpu().tolist()[0] > 0
