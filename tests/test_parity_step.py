@@ -90,3 +90,32 @@ def test_step_with_one_phase_only():
                        num_splits=dw.num_splits)
     torch.cuda.synchronize()
     assert D["count"].cpu().tolist()[0] > 0
+
+
+def test_step_replayed_from_a_cuda_graph_equals_eager():
+    pw, dw, px, dx, P, D = make_case()
+    factors = {"prefill": 100.0, "decode": 50.0}
+    run_step(pw, dw, P, D, factors)
+    eager = [P["o"].clone(), P["lse"].clone(), D["o"].clone(), D["lse"].clone(),
+             P["count"].clone(), D["count"].clone()]
+    for t in (P["o"], D["o"]):
+        t.zero_()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm-up outside capture (attributes, descriptors)
+        sk.sskip_attn_step(threshold_scale_factor=factors, sm_scale=pw.scale, prefill=P,
+                           decode=D, num_splits=dw.num_splits)
+    torch.cuda.current_stream().wait_stream(s)
+    with torch.cuda.graph(g):
+        sk.sskip_attn_step(threshold_scale_factor=factors, sm_scale=pw.scale, prefill=P,
+                           decode=D, num_splits=dw.num_splits)
+    for t in (P["o"], D["o"], P["count"], D["count"]):
+        t.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert sk.sskip_get_status() == sk.SSKIP_OK
+    got = [P["o"], P["lse"], D["o"], D["lse"], P["count"], D["count"]]
+    for a, b in zip(got, eager):
+        assert torch.equal(a, b)
+    del g
