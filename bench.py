@@ -893,7 +893,7 @@ def main(argv=None):
     ap.add_argument("--warp-vote-readings", default="lit,rms",
                     help="readings also timed with the per-warp (32-row) vote; '' for none")
     ap.add_argument("--sweep", action="store_true",
-                    help="threshold sweep of --prefill (default: the 128K long prefill)")
+                    help="threshold sweep of --prefill over 0, 100, 1000, 5000 (pass the 128K workload for the long-prefill sweep)")
     ap.add_argument("--calibrate", action="store_true",
                     help="calibrate the factors to --targets skip ratios and time them")
     ap.add_argument("--targets", default="0.25,0.5,0.75")
