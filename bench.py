@@ -10,12 +10,22 @@ One step = one pass of the whole hot path over one batch of synthetic input:
     lengths uniform in [16K, 32K], Bc=64, 16 splits, tsf=500) followed by the
     log-sum-exp merge.
 
+The prefill legs also run with the per-warp (32-row slice) vote.
+
 `value` is the prefill throughput in executed TFLOP/s (tensor work actually
 issued: 2 Br Bc d per visited tile for Q K^T plus 2 Br Bc d per kept tile for
 P V), over all ranks. Dense-equivalent TFLOP/s, skip fractions and the decode
-GB/s on bytes actually moved are reported beside it.
+GB/s on bytes actually moved are reported beside it. `e2e` is the same metric
+through the library's host-memory calls (sskip_attn_prefill_host, which
+overlaps the copies with the kernels, and sskip_attn_decode_host), pinned
+host inputs in and outputs out inside the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Other modes (one GPU): --sweep (speed vs skip over threshold factors),
+--calibrate (factors calibrated to target skip ratios), --reorder (video
+workload in raster vs Hilbert token order), --step (one serving step with a
+factor per phase, eager and CUDA-graph replay).
 
 For N > 1 launch under torch.distributed.run: every rank runs an independent
 replica (the method has no cross-GPU exchange), times are maxed over ranks.

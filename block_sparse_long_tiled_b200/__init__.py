@@ -1,9 +1,12 @@
 """Skip-Softmax tiled attention on B200 (sm_100a).
 
 Thin Python binding of libsskip_attn.so (C ABI in include/sskip_attn.h). The
-functions below only marshal torch tensors into the C calls of the same names:
-every step of the computation runs in the library's CUDA kernels. There is no
-CPU fallback; a missing library is an error.
+sskip_* functions below only marshal torch tensors into the C calls of the
+same names, and the conveniences after them only allocate outputs and chain
+those calls: every step of the computation runs in the library, in its CUDA
+kernels or, for the two host-side steps (the calibration's factor selection
+and the Hilbert order), in its C++. There is no CPU fallback; a missing
+library is an error.
 
 The method (TensorRT-LLM Skip-Softmax article, "Skip Softmax 的三步走算法"
 section): per attention tile, compare the tile's local maximum logit with the
