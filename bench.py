@@ -574,6 +574,7 @@ def run_sweep(args):
         q, k, v = td(x["q"]), td(x["k"]), td(x["v"])
         del x
         base_ms = None
+        hx = synth.prefill_inputs(w0, rd) if args.sweep_oracle else None
         for tsf in synth.LLAMA70B_TSF_SWEEP:
             w = w0.replace(tsf=tsf)
             out = sk.prefill(q, k, v, causal=w.causal, sm_scale=w.scale,
@@ -595,8 +596,18 @@ def run_sweep(args):
             base_ms = ms if tsf == 0 else base_ms
             f = prefill_flops(w, c[1], c[0])
             s = c[0] / max(1, c[1])
+            ora = {}
+            if hx is not None:
+                # The oracle on a stratified sample of whole query tiles,
+                # extrapolated to the call by executed FLOPs (labelled as such).
+                units = np.array([(0, h, i) for h in (0, w.Hq // 2)
+                                  for i in np.linspace(0, w.n_q - 1, 8).astype(int)], np.int32)
+                r = time_oracle(w, hx, units, os.cpu_count() or 1)
+                ora = {"oracle_sample_units": int(len(units)), "oracle_sample_s": r["seconds"],
+                       "oracle_extrapolated_s": r["seconds"] * f["executed"] / r["executed_flops"],
+                       "oracle_cores": os.cpu_count() or 1}
             print(json.dumps({"sweep": w.name, "reading": rd, "threshold_scale_factor": tsf,
-                              "ms": ms, "skip_fraction": s,
+                              **ora, "ms": ms, "skip_fraction": s,
                               "executed_tflops": f["executed"] / ms / 1e9,
                               "executed_frac_of_peak": f["executed"] / ms / 1e9 / peak,
                               "dense_equiv_tflops": f["dense"] / ms / 1e9,
@@ -904,6 +915,8 @@ def main(argv=None):
                     help="readings also timed with the per-warp (32-row) vote; '' for none")
     ap.add_argument("--sweep", action="store_true",
                     help="threshold sweep of --prefill over 0, 100, 1000, 5000 (pass the 128K workload for the long-prefill sweep)")
+    ap.add_argument("--sweep-oracle", action="store_true",
+                    help="with --sweep: time the CPU oracle on a sample and extrapolate")
     ap.add_argument("--calibrate", action="store_true",
                     help="calibrate the factors to --targets skip ratios and time them")
     ap.add_argument("--targets", default="0.25,0.5,0.75")
