@@ -108,3 +108,52 @@ def test_product_path_has_no_oracle_dependency():
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
                 assert "sskip_oracle" not in src, f
+
+
+def test_vote_record_and_host_entry_validation(lib):
+    P = ctypes.c_void_p
+    odd4 = P((1 << 20) + 2)  # not 4-byte aligned
+    # sskip_attn_prefill_vote: vote_rows must be Br or 32; records 4-byte aligned.
+    f = lib.sskip_attn_prefill_vote
+    args = [FAKE] * 5 + [1, 2, 1, 128, 128, 1, ctypes.c_float(0.088), ctypes.c_float(10.0), 128, 128]
+    assert f(*args, 48, None, None, None, None, None) == sk.SSKIP_ERR_UNSUPPORTED
+    assert f(*args, 64, None, None, None, None, None) == sk.SSKIP_ERR_UNSUPPORTED
+    assert f(*args, 32, None, None, None, odd4, None) == sk.SSKIP_ERR_INVALID_ARG
+    # sskip_attn_decode_crit: misaligned record.
+    g = lib.sskip_attn_decode_crit
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 8, 2, 256, 128, ctypes.c_float(0.088),
+             ctypes.c_float(5.0), 64, 4, FAKE, 1 << 30, None, None, odd4, None) == \
+        sk.SSKIP_ERR_INVALID_ARG
+    # sskip_attn_prefill_host: pointers, shapes and d are checked before any CUDA call.
+    h = lib.sskip_attn_prefill_host
+    tail = [ctypes.c_float(0.088), ctypes.c_float(10.0), 128, 128]
+    assert h(*([None] + [FAKE] * 9), 1, 2, 1, 128, 128, 1, *tail, 0, None, None) == \
+        sk.SSKIP_ERR_INVALID_ARG
+    assert h(*([FAKE] * 10), 1, 3, 2, 128, 128, 1, *tail, 0, None, None) == \
+        sk.SSKIP_ERR_INVALID_ARG
+    assert h(*([FAKE] * 10), 1, 2, 1, 128, 128, 1, *tail, -1, None, None) == \
+        sk.SSKIP_ERR_INVALID_ARG
+    assert h(*([FAKE] * 10), 1, 2, 1, 128, 96, 1, *tail, 0, None, None) == \
+        sk.SSKIP_ERR_UNSUPPORTED
+    # sskip_attn_decode_host: host and staging pointers.
+    dh = lib.sskip_attn_decode_host
+    assert dh(*([None] + [FAKE] * 9), 2, 8, 2, 256, 128, ctypes.c_float(0.088),
+              ctypes.c_float(5.0), 64, 4, FAKE, 1 << 30, None, None) == sk.SSKIP_ERR_INVALID_ARG
+    # sskip_permute_rows: in place, row size and index alignment.
+    pr = lib.sskip_permute_rows
+    assert pr(FAKE, FAKE, FAKE, 2, 64, 128, 0, None) == sk.SSKIP_ERR_INVALID_ARG
+    assert pr(FAKE, P(1 << 21), FAKE, 2, 64, 6, 0, None) == sk.SSKIP_ERR_INVALID_ARG
+    assert pr(FAKE, P(1 << 21), odd4, 2, 64, 128, 0, None) == sk.SSKIP_ERR_INVALID_ARG
+    assert pr(FAKE, P(1 << 21), FAKE, 0, 64, 128, 0, None) == sk.SSKIP_ERR_INVALID_ARG
+    # sskip_attn_step: at least one phase.
+    st = lib.sskip_attn_step
+    assert st(*([None] * 5), 0, 0, 1, 128, 128, None, *([None] * 6), 0, 0, 4, None, 0, None,
+              8, 2, 128, ctypes.c_float(0.088), ctypes.c_float(1000.0), ctypes.c_float(500.0),
+              None) == sk.SSKIP_ERR_INVALID_ARG
+    # sskip_calibrate_factor: bad ratio.
+    cf = lib.sskip_calibrate_factor
+    d = ctypes.c_double()
+    import numpy as np
+    c = np.zeros(4, np.float32)
+    assert cf(c.ctypes.data_as(P), 4, ctypes.c_double(1.5), ctypes.c_double(10.0),
+              ctypes.byref(d), None, None) == sk.SSKIP_ERR_INVALID_ARG
