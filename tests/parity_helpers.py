@@ -8,10 +8,15 @@ ln t - (m_local - m_run) is within NEAR_TIE of zero, where fp32 accumulation
 order decides. A unit with such a flip is checked against fp64 attention
 restricted to the GPU's own kept tiles (the closed form of the method), since
 both decisions are then correct readings of the same rule.
+
+Every check that forgives a flip records it in FLIP_LOG (test id, decisions
+compared, flips, largest |margin| among them); tests/conftest.py prints the
+log at the end of the run, so the gate can be set from what was measured.
 """
 from __future__ import annotations
 
 import math
+import os
 
 import numpy as np
 import torch
@@ -39,6 +44,21 @@ def check_counts(gpu_skipped: int, ora_skipped: int, gpu_visited: int, ora_visit
     assert abs(gpu_skipped - ora_skipped) <= COUNT_REL * ora_skipped, (gpu_skipped, ora_skipped)
 
 
+FLIP_LOG: list[dict] = []
+# |GPU critical value - fp64 closed form| per record check: how far the
+# kernels' decision quantity sits from the exact one.
+CRIT_LOG: list[dict] = []
+
+
+def note_flips(n_compared: int, flipped_margins) -> None:
+    """Record the decisions a test compared and the oracle margins of those
+    that flipped (already checked against NEAR_TIE by the caller)."""
+    m = np.abs(np.asarray(flipped_margins, np.float64)).ravel()
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    FLIP_LOG.append({"test": test, "compared": int(n_compared), "flips": int(m.size),
+                     "worst": float(m.max()) if m.size else 0.0})
+
+
 def check_tiles(gpu_state: np.ndarray, ora_state: np.ndarray, ora_margin: np.ndarray):
     """Returns the boolean mask of flipped tiles after asserting each is a near-tie."""
     diff = gpu_state != ora_state
@@ -47,6 +67,7 @@ def check_tiles(gpu_state: np.ndarray, ora_state: np.ndarray, ora_margin: np.nda
         assert np.all((gpu_state[diff] > 0) & (ora_state[diff] > 0)), "visit sets differ"
         worst = float(np.max(np.abs(ora_margin[diff])))
         assert worst < NEAR_TIE, f"{int(diff.sum())} decision flips, worst margin {worst}"
+    note_flips(int((ora_state > 0).sum()), ora_margin[diff])
     return diff
 
 

@@ -16,7 +16,7 @@ import torch
 import block_sparse_long_tiled_b200 as sk
 import oracle
 import synth
-from parity_helpers import COUNT_REL, NEAR_TIE, to_device
+from parity_helpers import COUNT_REL, CRIT_LOG, NEAR_TIE, note_flips, to_device
 from synth import DecodeWorkload, PrefillWorkload
 
 pytestmark = pytest.mark.gpu
@@ -51,6 +51,7 @@ def check_crit(gpu, ref):
     assert np.array_equal(np.isfinite(gpu), fin)
     d = np.abs(gpu[fin].astype(np.float64) - ref[fin])
     assert d.max() < NEAR_TIE, d.max()
+    CRIT_LOG.append({"compared": int(fin.sum()), "worst": float(d.max())})
 
 
 def gpu_prefill_crit(w, x):
@@ -114,6 +115,7 @@ def test_prefill_calibration_llama8b_16k():
         o_skip = ora["tile_state"][n] == 2
         flips = g_skip[:i + 1] != o_skip[:i + 1]
         assert np.all(np.abs(ora["tile_margin"][n][:i + 1][flips]) < NEAR_TIE)
+        note_flips(i + 1, ora["tile_margin"][n][:i + 1][flips])
 
 
 def decode_case():

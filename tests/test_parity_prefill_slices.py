@@ -15,7 +15,7 @@ import torch
 import block_sparse_long_tiled_b200 as sk
 import oracle
 import synth
-from parity_helpers import (COUNT_REL, NEAR_TIE, bf16_host, check_counts, check_rows,
+from parity_helpers import (COUNT_REL, NEAR_TIE, bf16_host, check_counts, check_rows, note_flips,
                             to_device, unit_slice_margins, unit_slice_restricted_reference)
 from synth import PrefillWorkload
 
@@ -55,13 +55,17 @@ def compare_units(w, x, g, ora, units, tsf):
         sm_o = ora["slice_mask"][n]
         assert np.array_equal(sm_g == 0, sm_o == 0), f"visit sets differ in {(b, hq, i)}"
         diff_bits = (sm_g ^ sm_o) & 0x7F
+        flipped = []
         if diff_bits.any():
             marg = unit_slice_margins(x, w, b, hq, i, R, tsf)
             for j in np.nonzero(diff_bits)[0]:
                 for s in range(w.Br // R):
                     if diff_bits[j] >> s & 1:
                         assert abs(marg[s, j]) < NEAR_TIE, (b, hq, i, j, s, marg[s, j])
+                        flipped.append(marg[s, j])
                         flips += 1
+        note_flips(int((sm_o != 0).sum()) * (w.Br // R), flipped)
+        if diff_bits.any():
             o_ref, lse_ref = unit_slice_restricted_reference(x, w, b, hq, i, sm_g, R)
         else:
             o_ref, lse_ref = ora["o"][n, :r1 - r0], ora["lse"][n, :r1 - r0]
