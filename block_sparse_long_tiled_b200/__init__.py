@@ -16,6 +16,7 @@ tile's softmax, its P.V and its V load; t = threshold_scale_factor / L
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -123,13 +124,46 @@ def _check(rc: int, what: str):
         raise SSkipError(rc, what)
 
 
-def _bf16_view(t):
+def _bf16_view(t, cuda: bool = True):
     # bf16 tensors, or raw bf16 bits stored as int16/uint16, are passed as is.
     if t.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
         raise TypeError(f"expected bf16 storage, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
+    if t.is_cuda != cuda:
+        raise ValueError(f"expected a {'CUDA' if cuda else 'host'} tensor")
     return t
+
+
+def _dev(t, dtype, what: str, cuda: bool = True):
+    """Check an optional non-bf16 argument: dtype, device side, contiguity."""
+    if t is None:
+        return t
+    if t.dtype != dtype:
+        raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if t.is_cuda != cuda:
+        raise ValueError(f"{what} must be a {'CUDA' if cuda else 'host'} tensor")
+    return t
+
+
+def _check_counts(t, n: int):
+    # Counters are unsigned 64-bit on the device; int64 storage of them is accepted.
+    if t is not None:
+        _dev(t, torch.int64, "skip_count")
+        if t.numel() < n:
+            raise ValueError(f"skip_count needs {n} entries")
+
+
+def _alloc_on(stream):
+    """Allocate on the stream a convenience launches on, so that buffers freed
+    when it returns are reused only after that stream's work."""
+    if stream is None:
+        return contextlib.nullcontext()
+    if not isinstance(stream, torch.cuda.Stream):
+        stream = torch.cuda.ExternalStream(int(stream))
+    return torch.cuda.stream(stream)
 
 
 def sskip_attn_prefill(q, k, v, o, lse, *, causal: bool, sm_scale: float,
@@ -140,6 +174,9 @@ def sskip_attn_prefill(q, k, v, o, lse, *, causal: bool, sm_scale: float,
     sskip_attn_prefill_ex."""
     for t in (q, k, v, o):
         _bf16_view(t)
+    _dev(lse, torch.float32, "lse")
+    _dev(tile_state, torch.uint8, "tile_state")
+    _check_counts(skip_count, 2)
     B, Hq, L, d = q.shape
     Hkv = k.shape[1]
     rc = lib().sskip_attn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv,
@@ -158,6 +195,11 @@ def sskip_attn_prefill_vote(q, k, v, o, lse, *, causal: bool, sm_scale: float,
     sskip_attn_prefill_vote."""
     for t in (q, k, v, o):
         _bf16_view(t)
+    _dev(lse, torch.float32, "lse")
+    _dev(tile_state, torch.uint8, "tile_state")
+    _dev(slice_mask, torch.uint8, "slice_mask")
+    _dev(tile_crit, torch.float32, "tile_crit")
+    _check_counts(counts, 4)
     B, Hq, L, d = q.shape
     Hkv = k.shape[1]
     rc = lib().sskip_attn_prefill_vote(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq,
@@ -173,10 +215,12 @@ def sskip_attn_prefill_host(host: dict, dev: dict, *, causal: bool, sm_scale: fl
                             kv_per_chunk: int = 0, skip_count=None, stream=None) -> None:
     """Marshal host tensors (q, k, v, o, lse; pinned for overlap) and device
     staging tensors of the same shapes into sskip_attn_prefill_host."""
-    for t in (host["q"], host["k"], host["v"], host["o"], dev["q"], dev["k"], dev["v"], dev["o"]):
-        _bf16_view(t)
-    if host["q"].is_cuda or not dev["q"].is_cuda:
-        raise ValueError("host tensors on the CPU, staging tensors on the GPU")
+    for n in ("q", "k", "v", "o"):
+        _bf16_view(host[n], cuda=False)
+        _bf16_view(dev[n])
+    _dev(host["lse"], torch.float32, "host lse", cuda=False)
+    _dev(dev["lse"], torch.float32, "lse")
+    _check_counts(skip_count, 2)
     B, Hq, L, d = host["q"].shape
     Hkv = host["k"].shape[1]
     rc = lib().sskip_attn_prefill_host(*(_ptr(host[n]) for n in ("q", "k", "v", "o", "lse")),
@@ -192,8 +236,16 @@ def sskip_attn_decode_host(host: dict, dev: dict, kcache, vcache, *, sm_scale: f
                            workspace=None, skip_count=None, stream=None) -> None:
     """Marshal host q, seqlens, o, lse (pinned for async copies), their device
     staging buffers and the device-resident caches into sskip_attn_decode_host."""
-    for t in (host["q"], host["o"], dev["q"], dev["o"], kcache, vcache):
+    for n in ("q", "o"):
+        _bf16_view(host[n], cuda=False)
+        _bf16_view(dev[n])
+    for t in (kcache, vcache):
         _bf16_view(t)
+    _dev(host["seqlens"], torch.int32, "host seqlens", cuda=False)
+    _dev(dev["seqlens"], torch.int32, "seqlens")
+    _dev(host["lse"], torch.float32, "host lse", cuda=False)
+    _dev(dev["lse"], torch.float32, "lse")
+    _check_counts(skip_count, 2)
     B, Hq, d = host["q"].shape
     Hkv, Lmax = kcache.shape[1], kcache.shape[2]
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -206,6 +258,16 @@ def sskip_attn_decode_host(host: dict, dev: dict, kcache, vcache, *, sm_scale: f
     _check(rc, "sskip_attn_decode_host")
 
 
+def _check_decode_args(q, kcache, vcache, seqlens, o, lse, skip_count):
+    for t in (q, kcache, vcache, o):
+        _bf16_view(t)
+    # int32 lengths on the device: an int64 tensor would be read as pairs of
+    # 32-bit words, i.e. wrong lengths.
+    _dev(seqlens, torch.int32, "seqlens")
+    _dev(lse, torch.float32, "lse")
+    _check_counts(skip_count, 2)
+
+
 def sskip_attn_decode_workspace_size(B: int, Hq: int, d: int, num_splits: int) -> int:
     return int(lib().sskip_attn_decode_workspace_size(B, Hq, d, num_splits))
 
@@ -215,8 +277,8 @@ def sskip_attn_decode(q, kcache, vcache, seqlens, o, lse, *, sm_scale: float,
                       workspace=None, skip_count=None, tile_state=None, stream=None) -> None:
     """Marshal q [B,Hq,d], caches [B,Hkv,Lmax,d] bf16, seqlens [B] int32,
     o [B,Hq,d] bf16, lse [B,Hq] fp32 and a uint8 workspace into sskip_attn_decode_ex."""
-    for t in (q, kcache, vcache, o):
-        _bf16_view(t)
+    _check_decode_args(q, kcache, vcache, seqlens, o, lse, skip_count)
+    _dev(tile_state, torch.uint8, "tile_state")
     B, Hq, d = q.shape
     Hkv, Lmax = kcache.shape[1], kcache.shape[2]
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -234,8 +296,9 @@ def sskip_attn_decode_crit(q, kcache, vcache, seqlens, o, lse, *, sm_scale: floa
                            stream=None) -> None:
     """sskip_attn_decode plus the fp32 critical-value record tile_crit
     [B, Hkv, ceil(Lmax/Bc)] (sskip_attn_decode_crit)."""
-    for t in (q, kcache, vcache, o):
-        _bf16_view(t)
+    _check_decode_args(q, kcache, vcache, seqlens, o, lse, skip_count)
+    _dev(tile_state, torch.uint8, "tile_state")
+    _dev(tile_crit, torch.float32, "tile_crit")
     B, Hq, d = q.shape
     Hkv, Lmax = kcache.shape[1], kcache.shape[2]
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -267,8 +330,7 @@ def sskip_attn_decode_noalloc(q, kcache, vcache, seqlens, o, lse, *, sm_scale: f
     sskip_attn_decode_noalloc: for callers that cannot allocate device memory,
     the library's own fixed scratch array (DECODE_NOALLOC_SCRATCH_BYTES) holds
     the split partials. Calls that overlap on the GPU race on that array."""
-    for t in (q, kcache, vcache, o):
-        _bf16_view(t)
+    _check_decode_args(q, kcache, vcache, seqlens, o, lse, skip_count)
     B, Hq, d = q.shape
     Hkv, Lmax = kcache.shape[1], kcache.shape[2]
     rc = lib().sskip_attn_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens),
@@ -294,20 +356,19 @@ def prefill(q, k, v, *, causal: bool, sm_scale: float, threshold_scale_factor: f
     with ``vote_rows`` (Br or 32), run sskip_attn_prefill_vote instead and
     also return the four counters and the slice record."""
     B, Hq, L, d = q.shape
-    o = torch.empty((B, Hq, L, d), dtype=q.dtype, device=q.device)
-    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
-    tiles = None
     rec_shape = (B, Hq, -(-L // Br), -(-L // Bc))
-    if with_tiles:
-        tiles = torch.empty(rec_shape, dtype=torch.uint8, device=q.device)
+    with _alloc_on(stream):
+        o = torch.empty((B, Hq, L, d), dtype=q.dtype, device=q.device)
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+        tiles = torch.empty(rec_shape, dtype=torch.uint8, device=q.device) if with_tiles else None
+        counts = torch.zeros(2 if vote_rows is None else 4, dtype=torch.int64, device=q.device)
+        smask = (torch.empty(rec_shape, dtype=torch.uint8, device=q.device)
+                 if with_tiles and vote_rows is not None else None)
     if vote_rows is None:
-        counts = torch.zeros(2, dtype=torch.int64, device=q.device)
         sskip_attn_prefill(q, k, v, o, lse, causal=causal, sm_scale=sm_scale,
                            threshold_scale_factor=threshold_scale_factor, Br=Br, Bc=Bc,
                            skip_count=counts, tile_state=tiles, stream=stream)
         return {"o": o, "lse": lse, "counts": counts, "tile_state": tiles}
-    counts = torch.zeros(4, dtype=torch.int64, device=q.device)
-    smask = torch.empty(rec_shape, dtype=torch.uint8, device=q.device) if with_tiles else None
     sskip_attn_prefill_vote(q, k, v, o, lse, causal=causal, sm_scale=sm_scale,
                             threshold_scale_factor=threshold_scale_factor, Br=Br, Bc=Bc,
                             vote_rows=vote_rows, counts=counts, tile_state=tiles,
@@ -320,14 +381,14 @@ def decode(q, kcache, vcache, seqlens, *, sm_scale: float, threshold_scale_facto
     """Allocate outputs and workspace with torch and run sskip_attn_decode."""
     B, Hq, d = q.shape
     Hkv, Lmax = kcache.shape[1], kcache.shape[2]
-    o = torch.empty((B, Hq, d), dtype=q.dtype, device=q.device)
-    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    ws = torch.empty(sskip_attn_decode_workspace_size(B, Hq, d, num_splits), dtype=torch.uint8,
-                     device=q.device)
-    counts = torch.zeros(2, dtype=torch.int64, device=q.device)
-    tiles = None
-    if with_tiles:
-        tiles = torch.empty((B, Hkv, -(-Lmax // Bc)), dtype=torch.uint8, device=q.device)
+    with _alloc_on(stream):
+        o = torch.empty((B, Hq, d), dtype=q.dtype, device=q.device)
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        ws = torch.empty(sskip_attn_decode_workspace_size(B, Hq, d, num_splits),
+                         dtype=torch.uint8, device=q.device)
+        counts = torch.zeros(2, dtype=torch.int64, device=q.device)
+        tiles = (torch.empty((B, Hkv, -(-Lmax // Bc)), dtype=torch.uint8, device=q.device)
+                 if with_tiles else None)
     sskip_attn_decode(q, kcache, vcache, seqlens, o, lse, sm_scale=sm_scale,
                       threshold_scale_factor=threshold_scale_factor, Bc=Bc, num_splits=num_splits,
                       workspace=ws, skip_count=counts, tile_state=tiles, stream=stream)
@@ -340,9 +401,11 @@ def calibrate_prefill(q, k, v, *, causal: bool, sm_scale: float, target_ratio: f
     then the host selection of the factor that skips target_ratio of the
     tiles. Returns factor, achieved_ratio, visited and the record."""
     B, Hq, L, d = q.shape
-    o = torch.empty_like(q)
-    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
-    crit = torch.empty((B, Hq, -(-L // Br), -(-L // Bc)), dtype=torch.float32, device=q.device)
+    with _alloc_on(stream):
+        o = torch.empty_like(q)
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+        crit = torch.empty((B, Hq, -(-L // Br), -(-L // Bc)), dtype=torch.float32,
+                           device=q.device)
     sskip_attn_prefill_vote(q, k, v, o, lse, causal=causal, sm_scale=sm_scale,
                             threshold_scale_factor=0.0, Br=Br, Bc=Bc, vote_rows=Br,
                             tile_crit=crit, stream=stream)
@@ -358,11 +421,12 @@ def calibrate_decode(q, kcache, vcache, seqlens, *, sm_scale: float, target_rati
     sequence, so every t_b = factor / seqlens[b] stays below 1)."""
     B, Hq, d = q.shape
     Hkv, Lmax = kcache.shape[1], kcache.shape[2]
-    o = torch.empty((B, Hq, d), dtype=q.dtype, device=q.device)
-    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    ws = torch.empty(sskip_attn_decode_workspace_size(B, Hq, d, num_splits), dtype=torch.uint8,
-                     device=q.device)
-    crit = torch.empty((B, Hkv, -(-Lmax // Bc)), dtype=torch.float32, device=q.device)
+    with _alloc_on(stream):
+        o = torch.empty((B, Hq, d), dtype=q.dtype, device=q.device)
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        ws = torch.empty(sskip_attn_decode_workspace_size(B, Hq, d, num_splits),
+                         dtype=torch.uint8, device=q.device)
+        crit = torch.empty((B, Hkv, -(-Lmax // Bc)), dtype=torch.float32, device=q.device)
     sskip_attn_decode_crit(q, kcache, vcache, seqlens, o, lse, sm_scale=sm_scale,
                            threshold_scale_factor=0.0, Bc=Bc, num_splits=num_splits,
                            workspace=ws, tile_crit=crit, stream=stream)
@@ -402,14 +466,16 @@ def prefill_reordered(q, k, v, perm, *, sm_scale: float, threshold_scale_factor:
     the Hilbert order): gather Q, K, V, run the kernel, scatter O and lse back
     to the original order. Every step runs in the library's kernels; the tile
     record, if asked for, is in the reordered frame."""
-    qp, kp, vp = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    with _alloc_on(stream):
+        qp, kp, vp = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     for a, b in ((q, qp), (k, kp), (v, vp)):
         sskip_permute_rows(a, b, perm, scatter=False, stream=stream)
     out = prefill(qp, kp, vp, causal=False, sm_scale=sm_scale,
                   threshold_scale_factor=threshold_scale_factor, Br=Br, Bc=Bc,
                   with_tiles=with_tiles, vote_rows=vote_rows, stream=stream)
-    o = torch.empty_like(out["o"])
-    lse = torch.empty_like(out["lse"])
+    with _alloc_on(stream):
+        o = torch.empty_like(out["o"])
+        lse = torch.empty_like(out["lse"])
     sskip_permute_rows(out["o"], o, perm, scatter=True, stream=stream)
     sskip_permute_rows(out["lse"].unsqueeze(-1), lse.unsqueeze(-1), perm, scatter=True,
                        stream=stream)

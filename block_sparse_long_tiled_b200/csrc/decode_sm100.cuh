@@ -130,7 +130,14 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int Lb = p.seqlens[b];
+  // seqlens[b] must lie in [1, Lmax]. A length outside that range is latched
+  // as an invalid argument and clamped to it, so no copy leaves the sequence's
+  // [Lmax, d] slab and no record index leaves [0, ceil(Lmax / Bc)); a length
+  // of 0 leaves every split empty.
+  const int Lraw = p.seqlens[b];
+  if ((Lraw < 1 || Lraw > p.Lmax) && tid == 0 && split == 0 && kvh == 0)
+    latch_status(kStatusInvalidArg);
+  const int Lb = min(max(Lraw, 0), p.Lmax);
   const int n_k = (Lb + kDecBc - 1) / kDecBc;
   const int c_per = (n_k + p.S - 1) / p.S;
   const int j0 = split * c_per;
@@ -173,8 +180,22 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
     mbar_arrive_expect_tx(bar, bytes);
     bulk_load(ring + stage * L::kTileBytes, base + (size_t)(j0 + t) * kDecBc * D, bytes, bar);
   };
+  // Thread 0 issues every copy and keeps what an aborting CTA needs to wait
+  // them out before it exits: the number of K tiles issued (tiles go out in
+  // order) and, per V slot, whether it was used and the parity of its copies.
+  int k_issued = 0;
+  uint32_t v_used = 0, v_par = 0;
+  auto issue_k = [&](int t) {
+    issue(k_smem, t % kDecNK, kfull(t % kDecNK), kbase, t);
+    k_issued = t + 1;
+  };
+  auto issue_v = [&](int t) {
+    issue(v_smem, t % kDecNV, vfull(t % kDecNV), vbase, t);
+    v_used |= 1u << (t % kDecNV);
+    v_par ^= 1u << (t % kDecNV);
+  };
   if (tid == 0)
-    for (int t = 0; t < min(kDecNK, ntiles); ++t) issue(k_smem, t, kfull(t), kbase, t);
+    for (int t = 0; t < min(kDecNK, ntiles); ++t) issue_k(t);
 
   // Lane layout of the scores: 8 lanes per key (sub = lane % 8), 4 keys per
   // warp per pass; pass ps covers keys ps*32 + warp*4 + lane/8.
@@ -207,14 +228,19 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
   uint32_t v_phase = 0;      // one parity bit per V slot
   uint64_t kept_mask = 0;    // bit (t % 64): tile t was kept
   int n_skipped = 0;
+  // A bounded wait that gives up makes its warp stop work; the block leaves
+  // the tile loop together at the next barrier (__syncthreads_or).
+  bool bad = false;
+  bool aborted = false;
 
   for (int t = 0; t < ntiles + kDecLag; ++t) {
     float s[2] = {-INFINITY, -INFINITY};
     const bool live = t < ntiles;
-    if (live) {
+    if (live && !bad)
+      bad = !__all_sync(0xffffffffu, mbar_wait(kfull(t % kDecNK), (t / kDecNK) & 1, abort_flag));
+    if (live && !bad) {
       // ---- scores of this warp's 8 keys, in log2 units; keys past L_b -> -inf.
       const int ks = t % kDecNK;
-      mbar_wait(kfull(ks), (t / kDecNK) & 1, abort_flag);
       const int keys = tile_keys(t);
       const uint8_t* ktile = smem + L::kK + ks * L::kTileBytes;
       float mx = -INFINITY;
@@ -253,11 +279,14 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       if (kq == 0 && owner) wmax[((t & 1) * G + hs) * kDecWarps + warp] = mx;
     }
-    __syncthreads();  // maxima of tile t published; K slot t % NK free; P.V of t-1-LAG done
+    // maxima of tile t published; K slot t % NK free; P.V of t-1-LAG done
+    if (__syncthreads_or(bad)) {
+      aborted = true;
+      break;
+    }
 
     if (live) {
-      if (tid == 0 && t + kDecNK < ntiles && !*abort_flag)
-        issue(k_smem, (t + kDecNK) % kDecNK, kfull((t + kDecNK) % kDecNK), kbase, t + kDecNK);
+      if (tid == 0 && t + kDecNK < ntiles) issue_k(t + kDecNK);
       // ---- the joint decision, taken identically by every warp.
       const float* wm = wmax + ((t & 1) * G + hv) * kDecWarps;
       float m_loc = wm[0];
@@ -291,7 +320,7 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
         }
         if (lane < G) Abuf[(t % kDecNPB) * G + lane] = a;
         kept_mask |= 1ull << (t & 63);
-        if (tid == 0 && !*abort_flag) issue(v_smem, t % kDecNV, vfull(t % kDecNV), vbase, t);
+        if (tid == 0) issue_v(t);
       } else {
         kept_mask &= ~(1ull << (t & 63));
         n_skipped += 1;
@@ -304,9 +333,11 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
     if (u >= 0 && ((kept_mask >> (u & 63)) & 1)) {
       // ---- O = alpha O + P_u V_u over this warp's 8 keys.
       const int vs = u % kDecNV;
-      mbar_wait(vfull(vs), (v_phase >> vs) & 1, abort_flag);
+      bad = !__all_sync(0xffffffffu, mbar_wait(vfull(vs), (v_phase >> vs) & 1, abort_flag));
       v_phase ^= 1u << vs;
-      __syncwarp();
+    }
+    if (u >= 0 && ((kept_mask >> (u & 63)) & 1) && !bad) {
+      const int vs = u % kDecNV;
       const int keys = tile_keys(u);
       const float* Pu = Pbuf + (u % kDecNPB) * kDecKeysPerWarp * G;
       const uint8_t* vtile = smem + L::kV + vs * L::kTileBytes;
@@ -346,6 +377,29 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
         }
       }
     }
+  }
+
+  // A wait that gave up in the last tiles' P.V has met no barrier yet.
+  if (!aborted && __syncthreads_or(bad)) aborted = true;
+  if (aborted) {
+    // The split's result is unusable (the status word says why): publish an
+    // empty split, then wait out every copy still in flight before exiting.
+    for (int i = tid; i < G * D; i += kDecThreads)
+      p.o_part[((head0 + i / D) * p.S + split) * D + (i % D)] = 0.f;
+    if (tid < G) p.lse_part[(head0 + tid) * p.S + split] = -INFINITY;
+    if (tid == 0) {
+      int no_abort = 0;
+#pragma unroll
+      for (int s = 0; s < kDecNK; ++s)
+        if (k_issued > s) {  // the last K tile that went to slot s
+          const int t_last = s + (k_issued - 1 - s) / kDecNK * kDecNK;
+          mbar_wait(kfull(s), (t_last / kDecNK) & 1, &no_abort);
+        }
+#pragma unroll
+      for (int s = 0; s < kDecNV; ++s)  // the phase of the slot's last copy
+        if ((v_used >> s) & 1) mbar_wait(vfull(s), ((v_par >> s) & 1) ^ 1, &no_abort);
+    }
+    return;
   }
 
   // ---- epilogue: merge the warps' partial O and row sums, write the split.
@@ -410,9 +464,11 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    if (threadIdx.x == 0) lse_s = mx + __logf(sum);
+    // Every split empty (a sequence of length 0, or aborted splits): O = 0
+    // and lse = -inf rather than 0 / 0.
+    if (threadIdx.x == 0) lse_s = sum > 0.f ? mx + __logf(sum) : -INFINITY;
     __syncwarp();
-    const float inv = 1.f / sum;
+    const float inv = sum > 0.f ? 1.f / sum : 0.f;
     for (int s = threadIdx.x; s < p.S; s += 32) w_s[s] *= inv;
   }
   __syncthreads();

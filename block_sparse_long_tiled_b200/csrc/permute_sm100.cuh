@@ -20,8 +20,6 @@
 
 namespace sskip {
 
-constexpr int kStatusBadIndex = 1;  // SSKIP_ERR_INVALID_ARG latched by the device
-
 template <typename Chunk>
 __global__ void __launch_bounds__(256)
     permute_rows_kernel(const Chunk* __restrict__ src, Chunk* __restrict__ dst,
@@ -37,7 +35,7 @@ __global__ void __launch_bounds__(256)
     const int e = (int)(rem - (long long)i * chunks_per_row);
     const int j = __ldg(idx + i);
     if (j < 0 || j >= L) {  // not a permutation of 0 .. L-1: record it, touch nothing
-      latch_status(kStatusBadIndex);
+      latch_status(kStatusInvalidArg);
       continue;
     }
     const long long a = (m * L + i) * chunks_per_row + e;   // position i

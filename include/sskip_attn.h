@@ -35,7 +35,8 @@
  *    sskip_hilbert3d_order are host-only and synchronous.
  *  - The return value reports argument validation and launch errors
  *    synchronously (sskip_status).  Errors found on the device while a kernel
- *    runs (a bounded wait that ran out) are latched in a per-device status
+ *    runs (a bounded wait that ran out, an out-of-range device-side length
+ *    or index) are latched in a per-device status
  *    word that sskip_get_status() reads.  No C++ exception crosses this ABI.
  *  - Outputs, the counters included, are overwritten, never accumulated.
  */
@@ -160,6 +161,9 @@ int sskip_attn_prefill_vote(const void* q, const void* k, const void* v, void* o
  * The call returns after enqueueing; the outputs are in host memory once
  * `stream` has completed (it waits for the last copy).  The two copy streams
  * are created on first use, once per device, and kept for the process's life.
+ * Every argument check runs before the first copy; if an error is returned
+ * after copies were enqueued, `stream` still waits for all of them, so the
+ * buffers may be reused in stream order.
  */
 int sskip_attn_prefill_host(const void* q_h, const void* k_h, const void* v_h, void* o_h,
                             float* lse_h, void* q_d, void* k_d, void* v_d, void* o_d, float* lse_d,
@@ -177,7 +181,12 @@ int sskip_attn_prefill_host(const void* q_h, const void* k_h, const void* v_h, v
  *   kcache  [B, Hkv, Lmax, d] bf16         lse [B, Hq] fp32 natural log
  *   vcache  [B, Hkv, Lmax, d] bf16             (written)
  *   seqlens [B] int32 on the device, 1 <= seqlens[b] <= Lmax; rows at or
- *           beyond seqlens[b] are never read.
+ *           beyond seqlens[b] are never read.  The host cannot see these
+ *           values, so the kernel checks them: a length outside [1, Lmax]
+ *           latches SSKIP_ERR_INVALID_ARG in the device status word (read it
+ *           with sskip_get_status) and is clamped into [0, Lmax] before use,
+ *           so no access leaves the sequence's cache slab; a clamped length
+ *           of 0 gives O = 0 and lse = -inf for that sequence's heads.
  *
  *   A decode tile is the G = Hq / Hkv query heads that share one kv head
  *   times Bc keys; the G heads take ONE joint decision, so a skipped tile
@@ -364,9 +373,11 @@ int sskip_permute_rows(const void* src, void* dst, const int32_t* idx, long long
 /*
  * Synchronises `stream`, then returns and clears the current device's status
  * word: SSKIP_OK, or the first device-side error latched since the last call
- * (SSKIP_ERR_TIMEOUT when a bounded wait inside a kernel ran out; the kernel
- * then abandoned its work and its outputs are undefined).  Returns
- * SSKIP_ERR_CUDA if the synchronisation itself failed.
+ * (SSKIP_ERR_TIMEOUT when a bounded wait inside a kernel ran out: the kernel
+ * then abandoned its work, waited out its own copies in flight and left its
+ * outputs undefined; SSKIP_ERR_INVALID_ARG when a decode length or a permute
+ * index held in device memory was out of range).  Returns SSKIP_ERR_CUDA if
+ * the synchronisation itself failed.
  */
 int sskip_get_status(void* stream);
 
