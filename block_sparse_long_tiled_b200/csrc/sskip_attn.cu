@@ -153,11 +153,12 @@ SSKIP_API int sskip_device_supported(int device) {
 namespace sskip {
 namespace {
 
-int prefill_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                 int Hkv, int L, int d, int causal, float sm_scale, float threshold_scale_factor,
-                 int Br, int Bc, int vote_rows, unsigned long long* counts, int n_counts,
-                 uint8_t* tile_state, uint8_t* slice_mask, float* tile_crit, void* stream,
-                 bool zero_counts = true) {
+// The synchronous argument checks of a prefill call (pointers, alignment,
+// shapes, scale and factor, supported tile sizes).
+int prefill_check(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  int B, int Hq, int Hkv, int L, int d, float sm_scale,
+                  float threshold_scale_factor, int Br, int Bc, int vote_rows,
+                  const unsigned long long* counts, const float* tile_crit) {
   if (!q || !k || !v || !o || !lse) return SSKIP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(counts) & 7u) ||
@@ -173,6 +174,18 @@ int prefill_impl(const void* q, const void* k, const void* v, void* o, float* ls
   const long long n_units = (L + kPfUnitRows - 1) / kPfUnitRows;
   if ((long long)B * Hq * n_units >= (1ll << 31) || (long long)B * Hq >= (1ll << 31))
     return SSKIP_ERR_UNSUPPORTED;
+  return SSKIP_OK;
+}
+
+int prefill_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                 int Hkv, int L, int d, int causal, float sm_scale, float threshold_scale_factor,
+                 int Br, int Bc, int vote_rows, unsigned long long* counts, int n_counts,
+                 uint8_t* tile_state, uint8_t* slice_mask, float* tile_crit, void* stream,
+                 bool zero_counts = true) {
+  const int rc = prefill_check(q, k, v, o, lse, B, Hq, Hkv, L, d, sm_scale,
+                               threshold_scale_factor, Br, Bc, vote_rows, counts, tile_crit);
+  if (rc != SSKIP_OK) return rc;
+  const long long n_units = (L + kPfUnitRows - 1) / kPfUnitRows;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   CUtensorMap mq, mk, mv;
@@ -640,11 +653,13 @@ SSKIP_API int sskip_attn_prefill_host(const void* q_h, const void* k_h, const vo
                                       int causal, float sm_scale, float threshold_scale_factor,
                                       int Br, int Bc, int kv_per_chunk,
                                       unsigned long long* skip_count, void* stream) {
-  if (!q_h || !k_h || !v_h || !o_h || !lse_h || !q_d || !k_d || !v_d || !o_d || !lse_d)
-    return SSKIP_ERR_INVALID_ARG;
-  if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Hq % Hkv != 0 || kv_per_chunk < 0)
-    return SSKIP_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return SSKIP_ERR_UNSUPPORTED;
+  if (!q_h || !k_h || !v_h || !o_h || !lse_h || kv_per_chunk < 0) return SSKIP_ERR_INVALID_ARG;
+  // Every check a chunk's prefill would make, before the first copy: the
+  // chunks' offsets keep the base pointers' alignment (a head's [L, d] bf16
+  // matrix is a multiple of 128 bytes, its lse row of 4).
+  int rc = prefill_check(q_d, k_d, v_d, o_d, lse_d, B, Hq, Hkv, L, d, sm_scale,
+                         threshold_scale_factor, Br, Bc, Br, skip_count, nullptr);
+  if (rc != SSKIP_OK) return rc;
   const int G = Hq / Hkv;
   const int n_units = (L + kPfUnitRows - 1) / kPfUnitRows;
   int kc = kv_per_chunk;
@@ -654,14 +669,15 @@ SSKIP_API int sskip_attn_prefill_host(const void* q_h, const void* k_h, const vo
   }
   kc = std::min(kc, Hkv);
   CopyStreams cs;
-  int rc = copy_streams(&cs);
+  rc = copy_streams(&cs);
   if (rc != SSKIP_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t row = (size_t)L * d * 2;  // bytes of one head's [L, d] bf16 matrix
   const int n_groups = (Hkv + kc - 1) / kc;
   const int n_chunks = B * n_groups;
-  // ev[2c]: chunk c copied in; ev[2c + 1]: chunk c computed; then start, end.
-  std::vector<cudaEvent_t> ev(2 * n_chunks + 2, nullptr);
+  // ev[2c]: chunk c copied in; ev[2c + 1]: chunk c computed; then start, the
+  // end of the copies out and the end of the copies in.
+  std::vector<cudaEvent_t> ev(2 * n_chunks + 3, nullptr);
   for (auto& e : ev)
     if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
       rc = SSKIP_ERR_CUDA;
@@ -706,10 +722,16 @@ SSKIP_API int sskip_attn_prefill_host(const void* q_h, const void* k_h, const vo
         !d2h(lse_h, lse_d, lo, ln))
       rc = SSKIP_ERR_CUDA;
   }
-  // The caller's stream completes only after the last copy out.
-  if (rc == SSKIP_OK && (cudaEventRecord(ev[2 * n_chunks + 1], cs.out) != cudaSuccess ||
-                         cudaStreamWaitEvent(st, ev[2 * n_chunks + 1], 0) != cudaSuccess))
-    rc = SSKIP_ERR_CUDA;
+  // The caller's stream completes only after every copy this call enqueued,
+  // on an error path as well: a caller that frees or reuses the buffers after
+  // an error must not race with copies still in flight.
+  if (ev[2 * n_chunks + 2]) {
+    const bool joined = cudaEventRecord(ev[2 * n_chunks + 1], cs.out) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, ev[2 * n_chunks + 1], 0) == cudaSuccess &&
+                        cudaEventRecord(ev[2 * n_chunks + 2], cs.in) == cudaSuccess &&
+                        cudaStreamWaitEvent(st, ev[2 * n_chunks + 2], 0) == cudaSuccess;
+    if (!joined && rc == SSKIP_OK) rc = SSKIP_ERR_CUDA;
+  }
   for (auto& e : ev)
     if (e) cudaEventDestroy(e);  // released once the recorded work completes
   return rc;
