@@ -83,6 +83,15 @@ constexpr int kPfVoteSlots = 4;
 #ifndef SSKIP_PF_NACC
 #define SSKIP_PF_NACC 4       // independent packed accumulators of the row sum
 #endif
+#ifndef SSKIP_PF_SPLIT_S
+#define SSKIP_PF_SPLIT_S 0    // S(j+1) as two halves, the upper one issued before P(j) is done
+#endif
+#ifndef SSKIP_PF_ROUNDED_L
+#define SSKIP_PF_ROUNDED_L 0  // 1: O is divided by the sum of the bf16 P that P.V used
+#endif
+#ifndef SSKIP_PF_MMA_NAP
+#define SSKIP_PF_MMA_NAP 0    // ns the MMA thread sleeps after a poll that found nothing to issue
+#endif
 #ifndef SSKIP_PF_FMA_EXP_D64
 #define SSKIP_PF_FMA_EXP_D64 SSKIP_PF_FMA_EXP  // the same, for head dim 64
 #endif
@@ -114,13 +123,14 @@ struct PrefillCfg {
   static constexpr int kK = kQ + 2 * kQBytes;
   static constexpr int kV = kK + kNK * kKVBytes;
   static constexpr int kBar = kV + kNV * kKVBytes;
-  // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], s_full[2],
-  // dec[2], vote_full[2][VS], vote_empty[2][VS], mma_done
-  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 2 + 2 + 4 * kPfVoteSlots + 1;
+  // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], then per
+  // warpgroup s_full, vote_mma, p_lo, s_hi_free, p_hi, then
+  // vote_full[2][VS], vote_empty[2][VS], mma_done
+  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 5 * 2 + 4 * kPfVoteSlots + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
-  // dec_kept[2], vote_kept[VS][2], warp vote flags [2 wg][2 parity][4], tmem, abort,
-  // warp gaps [2 wg][2 parity][4] (fp32)
-  static constexpr int kMiscInts = 2 + 2 * kPfVoteSlots + 16 + 2 + 16;
+  // kept flags [2 wg][2 parity], vote_kept[VS][2], warp vote flags
+  // [2 wg][2 parity][4], tmem, abort, warp gaps [2 wg][2 parity][4] (fp32)
+  static constexpr int kMiscInts = 4 + 2 * kPfVoteSlots + 16 + 2 + 16;
   static constexpr int kTotal = kMisc + kMiscInts * 4;
   static constexpr int kAlloc = kTotal + 1024;  // room to align the base to 1 KB
   static constexpr int kTmemCols = (2 * BC + 2 * D) <= 256 ? 256 : 512;
@@ -131,6 +141,21 @@ struct PrefillCfg {
 // EXT = false compiles the plain block vote with the tile_state record only;
 // EXT = true adds the per-warp vote, the slice and critical-value records and
 // the four counters (kept out of the plain kernel, which they slow down).
+//
+// Both contractions of a tile run as two halves of Bc/2 keys, so that the
+// tensor core never waits for a whole softmax step (S and P share the
+// Bc TMEM columns of a query tile; P of key tile j, bf16, fills the first
+// Bc/2 columns):
+//   S_hi(j+1) = Q K_{j+1}[Bc/2:]^T  as soon as the softmax has re-read the
+//                                    upper S columns of tile j;
+//   O += P_lo(j) V_j[:Bc/2]         as soon as P of the first half is stored;
+//   O += P_hi(j) V_j[Bc/2:], then S_lo(j+1) = Q K_{j+1}[:Bc/2]^T
+//                                    when the whole P(j) is stored.
+// Only the last pair sits between two softmax steps of a query tile.  A
+// skipped tile releases its S columns right after the vote and the next S
+// follows at once.  tcgen05 MMAs of one thread complete in issue order, so
+// S_lo(j+1) (issued after P.V(j)) is the commit that makes S(j+1) and O
+// visible together.
 template <int D, int BR, int BC, bool CAUSAL, bool EXT>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -139,7 +164,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   constexpr int NK = C::kNK, NV = C::kNV, VS = kPfVoteSlots;
   constexpr int NGRP = 128 / BR;  // vote groups per 128-row MMA tile
   constexpr int WPG = BR / 32;    // warps per vote group
+  constexpr int HK = BC / 2;      // keys per half tile
+  constexpr int HP = HK / 2;      // packed bf16 P columns per half tile
+  constexpr bool SPLIT = SSKIP_PF_SPLIT_S != 0;
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BC, 0, 0);
+  constexpr uint32_t IDESC_SH = idesc_bf16_f32(128, HK, 0, 0);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
   static_assert(BR == 64 || BR == 128, "Br");
   static_assert(BC == 64 || BC == 128, "Bc");
@@ -149,25 +178,29 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBar);
   int* misc = reinterpret_cast<int*>(smem + C::kMisc);
-  volatile int* dec_kept = misc;             // [2]
-  volatile int* vote_kept = misc + 2;        // [VS][2]
-  int* wflag = misc + 2 + 2 * VS;            // [2 wg][2 parity][4 warps]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 2 + 2 * VS + 16);
-  volatile int* abort_flag = misc + 2 + 2 * VS + 17;
-  float* wgap = reinterpret_cast<float*>(misc + 2 + 2 * VS + 18);  // [2 wg][2 parity][4 warps]
+  volatile int* kflag = misc;                // [2 wg][2 parity]
+  volatile int* vote_kept = misc + 4;        // [VS][2]
+  int* wflag = misc + 4 + 2 * VS;            // [2 wg][2 parity][4 warps]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 4 + 2 * VS + 16);
+  volatile int* abort_flag = misc + 4 + 2 * VS + 17;
+  float* wgap = reinterpret_cast<float*>(misc + 4 + 2 * VS + 18);  // [2 wg][2 parity][4 warps]
 
   const uint32_t b_qfull = smem_u32(&bars[0]);
   auto b_kfull = [&](int s) { return smem_u32(&bars[1 + s]); };
   auto b_kempty = [&](int s) { return smem_u32(&bars[1 + NK + s]); };
   auto b_vfull = [&](int s) { return smem_u32(&bars[1 + 2 * NK + s]); };
   auto b_vempty = [&](int s) { return smem_u32(&bars[1 + 2 * NK + NV + s]); };
-  auto b_sfull = [&](int w) { return smem_u32(&bars[1 + 2 * NK + 2 * NV + w]); };
-  auto b_dec = [&](int w) { return smem_u32(&bars[1 + 2 * NK + 2 * NV + 2 + w]); };
-  auto b_vote_full = [&](int w, int s) { return smem_u32(&bars[1 + 2 * NK + 2 * NV + 4 + w * VS + s]); };
+  constexpr int kWgBar = 1 + 2 * NK + 2 * NV;
+  auto b_sfull = [&](int w) { return smem_u32(&bars[kWgBar + w]); };      // MMA -> softmax
+  auto b_vmma = [&](int w) { return smem_u32(&bars[kWgBar + 2 + w]); };  // decision -> MMA
+  auto b_plo = [&](int w) { return smem_u32(&bars[kWgBar + 4 + w]); };   // P_lo stored
+  auto b_hfree = [&](int w) { return smem_u32(&bars[kWgBar + 6 + w]); }; // upper S re-read
+  auto b_phi = [&](int w) { return smem_u32(&bars[kWgBar + 8 + w]); };   // P_hi stored
+  auto b_vote_full = [&](int w, int s) { return smem_u32(&bars[kWgBar + 10 + w * VS + s]); };
   auto b_vote_empty = [&](int w, int s) {
-    return smem_u32(&bars[1 + 2 * NK + 2 * NV + 4 + 2 * VS + w * VS + s]);
+    return smem_u32(&bars[kWgBar + 10 + 2 * VS + w * VS + s]);
   };
-  const uint32_t b_mmadone = smem_u32(&bars[1 + 2 * NK + 2 * NV + 4 + 4 * VS]);
+  const uint32_t b_mmadone = smem_u32(&bars[kWgBar + 10 + 4 * VS]);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -199,7 +232,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     mbar_init(b_qfull, 1);
     for (int s = 0; s < NK; ++s) { mbar_init(b_kfull(s), 1); mbar_init(b_kempty(s), 1); }
     for (int s = 0; s < NV; ++s) { mbar_init(b_vfull(s), 1); mbar_init(b_vempty(s), 1); }
-    for (int w = 0; w < 2; ++w) { mbar_init(b_sfull(w), 1); mbar_init(b_dec(w), 1); }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(b_sfull(w), 1);
+      mbar_init(b_vmma(w), 1);
+      mbar_init(b_plo(w), 4);    // one arrival per softmax warp
+      mbar_init(b_hfree(w), 4);
+      mbar_init(b_phi(w), 4);
+    }
     for (int w = 0; w < 2; ++w)
       for (int s = 0; s < VS; ++s) { mbar_init(b_vote_full(w, s), 1); mbar_init(b_vote_empty(w, s), 1); }
     mbar_init(b_mmadone, 1);
@@ -253,90 +292,126 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint64_t dq0 = smem_desc_sw128(sbase + C::kQ, 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(sbase + C::kK, 16, 1024);
       const uint64_t dv0 = smem_desc_sw128(sbase + C::kV, BC * 128, 1024);
-      auto issue_s = [&](int w, int j) {
+      // Keys [k0, k0 + n) of S(w, j), n = Bc or Bc / 2, from key rows
+      // [k0, k0 + n) of the K tile (whole 1 KB swizzle atoms).
+      auto issue_s = [&](int w, int j, int k0, uint32_t idesc) {
         const uint64_t da = dq0 + (uint64_t)((w * C::kQBytes) >> 4);
-        const uint64_t db = dk0 + (uint64_t)(((j % NK) * C::kKVBytes) >> 4);
-        const uint32_t d_tmem = tmem + w * BC;
+        const uint64_t db = dk0 + (uint64_t)(((j % NK) * C::kKVBytes + k0 * 128) >> 4);
+        const uint32_t d_tmem = tmem + w * BC + k0;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oa = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
           const uint32_t ob = ((kk >> 2) * (BC * 128) + (kk & 3) * 32) >> 4;
-          umma_ss(d_tmem, da + oa, db + ob, IDESC_S, kk > 0 ? 1u : 0u);
+          umma_ss(d_tmem, da + oa, db + ob, idesc, kk > 0 ? 1u : 0u);
         }
-        umma_commit(b_sfull(w));
       };
       int pv_count[2] = {0, 0};
-      auto issue_pv = [&](int w, int vs) {
+      // O(w) += P(w)[:, half h] V[half h] from V slot vs; P read from TMEM.
+      auto issue_pv_half = [&](int w, int vs, int h) {
         const uint32_t p_tmem = tmem + w * BC;
         const uint32_t o_tmem = tmem + 2 * BC + w * D;
         const uint64_t dv = dv0 + (uint64_t)((vs * C::kKVBytes) >> 4);
-        const uint32_t acc0 = pv_count[w] > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < BC / 16; ++kk)
-          umma_ts(o_tmem, p_tmem + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), IDESC_PV,
-                  kk > 0 ? 1u : acc0);
-        ++pv_count[w];
+        for (int k2 = 0; k2 < HK / 16; ++k2) {
+          const int kk = h * (HK / 16) + k2;
+          const uint32_t acc = (kk > 0 || pv_count[w] > 0) ? 1u : 0u;
+          umma_ts(o_tmem, p_tmem + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), IDESC_PV, acc);
+        }
+        if (h == 1) ++pv_count[w];
       };
+      const int n_w[2] = {n_a, n_b};
+      int kc_w[2] = {0, 0};  // kept tiles per warpgroup: parity of p_lo / s_hi_free / p_hi
       bool ok = mbar_wait(b_qfull, 0, abort_flag);
       if (ok && n_j > 0) {
         ok = mbar_wait(b_kfull(0), 0, abort_flag);
         tc_fence_after();
         if (ok) {
-          if (n_a > 0) issue_s(0, 0);
-          if (n_b > 0) issue_s(1, 0);
+#pragma unroll
+          for (int w = 0; w < 2; ++w)
+            if (n_w[w] > 0) {
+              issue_s(w, 0, 0, IDESC_S);
+              umma_commit(b_sfull(w));
+            }
           umma_commit(b_kempty(0));
         }
       }
+      // Key tile j, warpgroup A then B: the decision; for a kept tile P_lo V
+      // as soon as P_lo is stored and P_hi V once P is complete; then
+      // S(j+1) (with the split option, its upper half as soon as the upper S
+      // columns of tile j have been re-read).  V_j goes to slot (number of
+      // earlier tiles some warpgroup kept) % NV, the V producer's numbering.
       int kc = 0;
       for (int j = 0; ok && j < n_j; ++j) {
         const int vs = kc % NV;
-        bool ka = false, kb = false, v_ready = false;
-        if (j < n_a) {
-          if (!mbar_wait(b_dec(0), j & 1, abort_flag)) break;
-          tc_fence_after();
-          ka = dec_kept[0] != 0;
-          if (ka) {
-            if (!mbar_wait(b_vfull(vs), (kc / NV) & 1, abort_flag)) break;
-            tc_fence_after();
-            v_ready = true;
-            issue_pv(0, vs);
-          }
-        }
         const bool nxt = j + 1 < n_j;
-        if (nxt) {
-          if (!mbar_wait(b_kfull((j + 1) % NK), ((j + 1) / NK) & 1, abort_flag)) break;
-          tc_fence_after();
-          if (j + 1 < n_a) issue_s(0, j + 1);
-        }
-        if (j < n_b) {
-          if (!mbar_wait(b_dec(1), j & 1, abort_flag)) break;
-          tc_fence_after();
-          kb = dec_kept[1] != 0;
-          if (kb) {
+        bool any_kept = false, v_ready = false, k_ready = false;
+        // K_{j+1} is waited for just before its first use, so that a late
+        // K tile never holds back a P.V.
+        auto need_k = [&]() {
+          if (!k_ready) k_ready = mbar_wait(b_kfull((j + 1) % NK), ((j + 1) / NK) & 1, abort_flag);
+          return k_ready;
+        };
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (j >= n_w[w]) continue;
+          const bool s_next = j + 1 < n_w[w];
+          if (!mbar_wait(b_vmma(w), j & 1, abort_flag)) { ok = false; break; }
+          const bool kept = kflag[w * 2 + (j & 1)] != 0;
+          if (kept) {
+            any_kept = true;
+            const uint32_t par = kc_w[w] & 1;
+            if (!mbar_wait(b_plo(w), par, abort_flag)) { ok = false; break; }
             if (!v_ready) {
-              if (!mbar_wait(b_vfull(vs), (kc / NV) & 1, abort_flag)) break;
-              tc_fence_after();
+              if (!mbar_wait(b_vfull(vs), (kc / NV) & 1, abort_flag)) { ok = false; break; }
+              v_ready = true;
             }
-            issue_pv(1, vs);
+            tc_fence_after();
+            issue_pv_half(w, vs, 0);
+            if (SPLIT && s_next) {
+              if (!mbar_wait(b_hfree(w), par, abort_flag) || !need_k()) { ok = false; break; }
+              tc_fence_after();
+              issue_s(w, j + 1, HK, IDESC_SH);
+            }
+            if (!mbar_wait(b_phi(w), par, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv_half(w, vs, 1);
+            ++kc_w[w];
+            if (s_next) {
+              if (!need_k()) { ok = false; break; }
+              issue_s(w, j + 1, 0, SPLIT ? IDESC_SH : IDESC_S);
+            }
+          } else if (s_next) {
+            if (!need_k()) { ok = false; break; }
+            tc_fence_after();
+            if constexpr (SPLIT) {
+              issue_s(w, j + 1, HK, IDESC_SH);
+              issue_s(w, j + 1, 0, IDESC_SH);
+            } else {
+              issue_s(w, j + 1, 0, IDESC_S);
+            }
           }
+          if (s_next) umma_commit(b_sfull(w));
         }
-        if (ka || kb) {
+        if (!ok) break;
+        if (any_kept) {
           umma_commit(b_vempty(vs));
           ++kc;
         }
-        if (nxt) {
-          if (j + 1 < n_b) issue_s(1, j + 1);
-          umma_commit(b_kempty((j + 1) % NK));
-        }
+        if (nxt) umma_commit(b_kempty((j + 1) % NK));
       }
-      // Every MMA issued by this thread completes before the epilogue reads O.
+      // Every MMA issued by this thread completes before the epilogue reads O
+      // and before TMEM is released.
       umma_commit(b_mmadone);
+      int no_abort = 0;
+      mbar_wait(b_mmadone, 0, &no_abort);
     } else if (warp == 2 && lane == 0) {
       // ================= V producer: issues V_j on the FIRST keep vote =====
       // Each warpgroup posts its vote on tile j as soon as it has its row
       // maxima; the first "keep" starts the V_j load, so its latency hides
-      // behind that warpgroup's exponentials.  Both votes are consumed in
-      // order to keep the slots' phases exact.
+      // behind that warpgroup's exponentials.  Loads are numbered in tile
+      // order over the tiles some warpgroup kept and go to slot number % NV;
+      // a tile both skip costs nothing here.  Both votes are consumed in order
+      // to keep the vote slots' phases exact.
       tma_prefetch_desc(&tmV);
       int kc = 0, last = -1;
       for (int j = 0; j < n_j && !*abort_flag; ++j) {
@@ -408,7 +483,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const bool t_pos = p.t_positive != 0;
     const float scale = p.scale_log2;
 
-    float m_run = -INFINITY, m_ref = -INFINITY, l_run = 0.f;
+    // l_run sums P in fp32 (for lse); lr_run sums the bf16-rounded P that the
+    // P.V MMA applied, so that O / lr_run weighs V with weights summing to 1.
+    float m_run = -INFINITY, m_ref = -INFINITY, l_run = 0.f, lr_run = 0.f;
     long long n_vis = 0, n_skip = 0, n_svis = 0, n_sskip = 0;
 
     auto post_vote = [&](int j, bool kept) {  // elected thread only
@@ -416,6 +493,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (j >= VS) mbar_wait(b_vote_empty(wg, vslot), ((j / VS) - 1) & 1, abort_flag);
       vote_kept[vslot * 2 + wg] = kept ? 1 : 0;
       mbar_arrive(b_vote_full(wg, vslot));
+    };
+    // This warp's part of a signal counted once per softmax warp: its TMEM
+    // accesses are complete (the caller waited for them) and ordered before
+    // the MMA warp's next tcgen05 operation.
+    auto warp_signal = [&](uint32_t bar) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
     };
 
     for (int j = 0; j < n_j; ++j) {
@@ -464,6 +549,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int o = 16; o > 0; o >>= 1) gap = fmaxf(gap, __shfl_xor_sync(0xffffffffu, gap, o));
         if (lane == 0) wgap[(wg * 2 + (j & 1)) * 4 + wq] = gap;
       }
+      // Every warp's S loads are complete before this barrier, so after it
+      // the whole S(j) has been read once.
       tc_fence_before();
       named_bar_sync(bar_id, 128);
       bool g_kept[NGRP];
@@ -502,117 +589,119 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         ++n_svis;
         n_sskip += wall ? 1 : 0;
       }
-      if (elected) post_vote(j, tile_kept);
-
-      if (tile_kept) {
-        // Block vote: every row of a kept group updates.  Warp vote: only the
-        // rows of a warp slice that did not pass.
-        const bool mine = row_in && ((EXT && p.slice_vote) ? (gvis && !wall) : g_kept[grp]);
-        float alpha = 1.f;
-        bool rescale = false;
-        if (mine) {
-          const float m_new = fmaxf(m_run, m_loc);
-          m_run = m_new;
-          if (m_ref == -INFINITY) {
-            m_ref = m_new;  // first kept tile of the row: its O row is still zero
-          } else if (m_new - m_ref > kRescaleLog2) {
-            alpha = ex2_approx(m_ref - m_new);
-            m_ref = m_new;
-            rescale = true;
-            l_run *= alpha;
-          }
-        }
-        // P = exp2(S * scale - m_ref) for kept rows, 0 otherwise; bf16 pairs.
-        const uint64_t scale2 = f2pack(scale, scale);
-        const float nref = mine ? kPackBias - m_ref : -INFINITY;
-        const uint64_t nref2 = f2pack(nref, nref);
-        __syncwarp();
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float o32[32];
-            tmem_ld32(tO + c * 32, o32);
-            uint32_t w32[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) w32[i] = __float_as_uint(o32[i] * alpha);
-            tmem_st32(tO + c * 32, w32);
-          }
-        }
-        if (EXT && __all_sync(0xffffffffu, !mine)) {
-          // No row of this warp takes part (its slice or group skipped the
-          // tile, or it is padding): P = 0 without any exponential.
-          uint32_t z[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) z[i] = 0u;
-#pragma unroll
-          for (int h = 0; h < BC / 64; ++h) tmem_st32(tS + h * 32, z);
-        } else {
-          uint64_t sum2v[SSKIP_PF_NACC];
-#pragma unroll
-          for (int a = 0; a < SSKIP_PF_NACC; ++a) sum2v[a] = f2pack(0.f, 0.f);
-          float suma = 0.f, sumb = 0.f;
-#pragma unroll
-          for (int h = 0; h < BC / 64; ++h) {  // 64 keys -> 32 packed columns at a time
-            uint32_t pk[32];
-            float* sh = s;
-            uint32_t rr[64];
-            if constexpr (SSKIP_PF_RELOAD) {
-              // The row max is known; re-read this half of S (its columns are
-              // still intact: P of half h lands in columns [32h, 32h + 32)).
-              tmem_ld32_async(tS + h * 64, rr);
-              tmem_ld32_async(tS + h * 64 + 32, rr + 32);
-              tmem_wait_ld_tie64(rr);
-              sh = reinterpret_cast<float*>(rr) - h * 64;
-              if (need_mask) {
-#pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                  const int key = key0 + h * 64 + c;
-                  if (key >= p.L || (CAUSAL && key > row)) rr[c] = __float_as_uint(-INFINITY);
-                }
-              }
-            }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int c = h * 32 + i;
-              float p0, p1;
-              if (SSKIP_PF_SCALAR && !exp2_on_fma<D>(c)) {
-                p0 = ex2_approx(fmaf(sh[2 * c], scale, nref));
-                p1 = ex2_approx(fmaf(sh[2 * c + 1], scale, nref));
-                suma += p0;
-                sumb += p1;
-              } else {
-                const uint64_t x2 = ffma2(f2pack(sh[2 * c], sh[2 * c + 1]), scale2, nref2);
-                if (exp2_on_fma<D>(c)) {
-                  f2unpack(exp2_fma2(x2), p0, p1);
-                } else {
-                  float x0, x1;
-                  f2unpack(x2, x0, x1);
-                  p0 = ex2_approx(x0);
-                  p1 = ex2_approx(x1);
-                }
-                sum2v[c % SSKIP_PF_NACC] = fadd2(sum2v[c % SSKIP_PF_NACC], f2pack(p0, p1));
-              }
-              if (SSKIP_PF_PACK_PRMT)
-                pk[i] = pack_bf16x2_halfup(p0, p1);
-              else
-                pk[i] = pack_bf16x2(p0, p1);
-            }
-            tmem_st32(tS + h * 32, pk);
-          }
-          uint64_t sum2 = sum2v[0];
-#pragma unroll
-          for (int a = 1; a < SSKIP_PF_NACC; ++a) sum2 = fadd2(sum2, sum2v[a]);
-          float sa, sb;
-          f2unpack(sum2, sa, sb);
-          l_run += mine ? ((sa + sb) + (suma + sumb)) : 0.f;
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        named_bar_sync(bar_id, 128);
-      }
       if (elected) {
-        dec_kept[wg] = tile_kept ? 1 : 0;
-        mbar_arrive(b_dec(wg));
+        post_vote(j, tile_kept);
+        kflag[wg * 2 + (j & 1)] = tile_kept ? 1 : 0;
+        mbar_arrive(b_vmma(wg));
+      }
+      if (!tile_kept) continue;
+
+      // Block vote: every row of a kept group updates.  Warp vote: only the
+      // rows of a warp slice that did not pass.
+      const bool mine = row_in && ((EXT && p.slice_vote) ? (gvis && !wall) : g_kept[grp]);
+      float alpha = 1.f;
+      bool rescale = false;
+      if (mine) {
+        const float m_new = fmaxf(m_run, m_loc);
+        m_run = m_new;
+        if (m_ref == -INFINITY) {
+          m_ref = m_new;  // first kept tile of the row: its O row is still zero
+        } else if (m_new - m_ref > kRescaleLog2) {
+          alpha = ex2_approx(m_ref - m_new);
+          m_ref = m_new;
+          rescale = true;
+          l_run *= alpha;
+          lr_run *= alpha;
+        }
+      }
+      // P = exp2(S * scale - m_ref) for kept rows, 0 otherwise; bf16 pairs.
+      const uint64_t scale2 = f2pack(scale, scale);
+      const float nref = mine ? kPackBias - m_ref : -INFINITY;
+      const uint64_t nref2 = f2pack(nref, nref);
+      __syncwarp();
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O(j-1) is complete: S(j) was committed after P.V(j-1).
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float o32[32];
+          tmem_ld32(tO + c * 32, o32);
+          uint32_t w32[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w32[i] = __float_as_uint(o32[i] * alpha);
+          tmem_st32(tO + c * 32, w32);
+        }
+      }
+      // No row of this warp takes part (its slice or group skipped the tile,
+      // or it is padding): P = 0 without any exponential.
+      const bool none = EXT && __all_sync(0xffffffffu, !mine);
+      uint64_t sum2v[SSKIP_PF_NACC], sumr2v[SSKIP_PF_NACC];
+#pragma unroll
+      for (int a = 0; a < SSKIP_PF_NACC; ++a) sum2v[a] = sumr2v[a] = f2pack(0.f, 0.f);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // HK keys -> HP packed columns at a time
+        uint32_t pk[HP];
+        if (none) {
+#pragma unroll
+          for (int i = 0; i < HP; ++i) pk[i] = 0u;
+          if (SPLIT && h == 1) warp_signal(b_hfree(wg));  // its S was read in the max pass
+        } else {
+          // The row max is known; re-read this half of S (its columns are
+          // still intact: P of half h lands in columns [h HP, h HP + HP)).
+          uint32_t rr[HK];
+          tmem_ld32_async(tS + h * HK, rr);
+          if constexpr (HK == 64) {
+            tmem_ld32_async(tS + h * HK + 32, rr + 32);
+            tmem_wait_ld_tie64(rr);
+          } else {
+            tmem_wait_ld_tie32(rr);
+          }
+          if (SPLIT && h == 1) warp_signal(b_hfree(wg));  // upper S columns free for S_hi(j+1)
+          const float* sh = reinterpret_cast<const float*>(rr);
+          if (need_mask) {
+#pragma unroll
+            for (int c = 0; c < HK; ++c) {
+              const int key = key0 + h * HK + c;
+              if (key >= p.L || (CAUSAL && key > row)) rr[c] = __float_as_uint(-INFINITY);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < HP; ++i) {
+            const int c = h * HP + i;  // pair index within the tile
+            float p0, p1;
+            const uint64_t x2 = ffma2(f2pack(sh[2 * i], sh[2 * i + 1]), scale2, nref2);
+            if (exp2_on_fma<D>(c)) {
+              f2unpack(exp2_fma2(x2), p0, p1);
+            } else {
+              float x0, x1;
+              f2unpack(x2, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            sum2v[c % SSKIP_PF_NACC] = fadd2(sum2v[c % SSKIP_PF_NACC], f2pack(p0, p1));
+            pk[i] = pack_bf16x2(p0, p1);
+            if (SSKIP_PF_ROUNDED_L)  // the two bf16 halves widened exactly
+              sumr2v[c % SSKIP_PF_NACC] =
+                  fadd2(sumr2v[c % SSKIP_PF_NACC], f2pack(__uint_as_float(pk[i] << 16),
+                                                          __uint_as_float(pk[i] & 0xFFFF0000u)));
+          }
+        }
+        if constexpr (HP == 32) tmem_st32(tS + h * HP, pk);
+        else tmem_st16(tS + h * HP, pk);
+        tmem_st_wait();
+        warp_signal(h == 0 ? b_plo(wg) : b_phi(wg));
+      }
+      if (!none) {
+        uint64_t sum2 = sum2v[0], sumr2 = sumr2v[0];
+#pragma unroll
+        for (int a = 1; a < SSKIP_PF_NACC; ++a) {
+          sum2 = fadd2(sum2, sum2v[a]);
+          sumr2 = fadd2(sumr2, sumr2v[a]);
+        }
+        float sa, sb;
+        f2unpack(sum2, sa, sb);
+        l_run += mine ? (sa + sb) : 0.f;
+        f2unpack(sumr2, sa, sb);
+        lr_run += mine ? (sa + sb) : 0.f;
       }
     }
 
@@ -622,7 +711,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     __syncwarp();
     const bool store = row_in && my_jmax >= 0 && n_own > 0 && l_run > 0.f;
     if (n_own > 0) {
-      const float inv_l = store ? 1.f / l_run : 0.f;
+      const float inv_l = store ? 1.f / (SSKIP_PF_ROUNDED_L ? lr_run : l_run) : 0.f;
       __nv_bfloat16* orow = p.o + (((size_t)b * p.Hq + hq) * p.L + (store ? row : 0)) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
