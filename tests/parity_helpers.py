@@ -27,7 +27,13 @@ MAX_ABS = 1e-2
 MEAN_ABS = 1e-3
 LSE_ABS = 1e-3
 COUNT_REL = 0.005
-NEAR_TIE = 1e-3
+# A decision can flip only where the fp32 oracle's margin and the kernel's own
+# decision quantity straddle zero. Measured: the oracle's fp32 margins lie
+# within 3.0e-6 of the fp64 closed form, the kernels' critical values within
+# 4.3e-6 of it (tests/test_parity_calibration.py records it), so a genuine
+# near-tie has |margin| < 7.3e-6; the gate is about 14 times that. No flip
+# was seen in 566,405 compared decisions.
+NEAR_TIE = 1e-4
 
 
 def to_device(bits: np.ndarray) -> torch.Tensor:

@@ -27,8 +27,8 @@ def _built():
     assert sk.lib().sskip_device_supported(torch.cuda.current_device()) == sk.SSKIP_OK
 
 
-def run_gpu(w, x, tsf=None):
-    q, k, v = to_device(x["q"]), to_device(x["k"]), to_device(x["v"])
+def run_gpu(w, x, tsf=None, dev=None):
+    q, k, v = dev if dev is not None else (to_device(x["q"]), to_device(x["k"]), to_device(x["v"]))
     out = sk.prefill(q, k, v, causal=w.causal, sm_scale=w.scale,
                      threshold_scale_factor=w.tsf if tsf is None else tsf, Br=w.Br, Bc=w.Bc,
                      with_tiles=True)
@@ -125,9 +125,9 @@ def sample_units(w, n, seed):
     return units
 
 
-def full_size_check(w, reading, n_units, tsf=None):
-    x = synth.prefill_inputs(w, reading)
-    g = run_gpu(w, x, tsf=tsf)
+def full_size_check(w, reading, n_units, tsf=None, x=None, dev=None):
+    x = synth.prefill_inputs(w, reading) if x is None else x
+    g = run_gpu(w, x, tsf=tsf, dev=dev)
     tsf = w.tsf if tsf is None else tsf
     units = sample_units(w, n_units, seed=w.seed)
     ora = oracle.prefill(x["q"], x["k"], x["v"], causal=w.causal, sm_scale=w.scale, tsf=tsf,
@@ -154,6 +154,13 @@ def test_videodit_prefill():
     full_size_check(synth.VIDEO_DIT_PREFILL, "lit", n_units=12)
 
 
-@pytest.mark.parametrize("tsf", synth.LLAMA70B_TSF_SWEEP)
-def test_llama70b_prefill_128k_sweep(tsf):
-    full_size_check(synth.LLAMA70B_PREFILL_128K, "rms", n_units=8, tsf=tsf)
+@pytest.mark.parametrize("reading", ["lit", "rms"])
+def test_llama70b_prefill_128k_sweep(reading):
+    # The 128K workload at every factor of its sweep, in the launch the
+    # benchmark times; 32 query tiles spread over the diagonal (plus both ends)
+    # are compared with the oracle at each factor.
+    w = synth.LLAMA70B_PREFILL_128K
+    x = synth.prefill_inputs(w, reading)
+    dev = (to_device(x["q"]), to_device(x["k"]), to_device(x["v"]))
+    for tsf in synth.LLAMA70B_TSF_SWEEP:
+        full_size_check(w, reading, n_units=32, tsf=tsf, x=x, dev=dev)
