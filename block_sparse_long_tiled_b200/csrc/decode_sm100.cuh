@@ -228,19 +228,19 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
   uint32_t v_phase = 0;      // one parity bit per V slot
   uint64_t kept_mask = 0;    // bit (t % 64): tile t was kept
   int n_skipped = 0;
-  // A bounded wait that gives up makes its warp stop work; the block leaves
-  // the tile loop together at the next barrier (__syncthreads_or).
-  bool bad = false;
-  bool aborted = false;
 
+  // A bounded wait that runs out raises the CTA's abort flag; from then on
+  // every wait returns at once, no new copy is issued and the loop runs out
+  // its remaining tiles on meaningless data (the outputs are undefined, the
+  // status word says why).  Copies already in flight are waited out after
+  // the loop.
   for (int t = 0; t < ntiles + kDecLag; ++t) {
     float s[2] = {-INFINITY, -INFINITY};
     const bool live = t < ntiles;
-    if (live && !bad)
-      bad = !__all_sync(0xffffffffu, mbar_wait(kfull(t % kDecNK), (t / kDecNK) & 1, abort_flag));
-    if (live && !bad) {
+    if (live) {
       // ---- scores of this warp's 8 keys, in log2 units; keys past L_b -> -inf.
       const int ks = t % kDecNK;
+      mbar_wait(kfull(ks), (t / kDecNK) & 1, abort_flag);
       const int keys = tile_keys(t);
       const uint8_t* ktile = smem + L::kK + ks * L::kTileBytes;
       float mx = -INFINITY;
@@ -279,14 +279,10 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       if (kq == 0 && owner) wmax[((t & 1) * G + hs) * kDecWarps + warp] = mx;
     }
-    // maxima of tile t published; K slot t % NK free; P.V of t-1-LAG done
-    if (__syncthreads_or(bad)) {
-      aborted = true;
-      break;
-    }
+    __syncthreads();  // maxima of tile t published; K slot t % NK free; P.V of t-1-LAG done
 
     if (live) {
-      if (tid == 0 && t + kDecNK < ntiles) issue_k(t + kDecNK);
+      if (tid == 0 && t + kDecNK < ntiles && !*abort_flag) issue_k(t + kDecNK);
       // ---- the joint decision, taken identically by every warp.
       const float* wm = wmax + ((t & 1) * G + hv) * kDecWarps;
       float m_loc = wm[0];
@@ -320,7 +316,7 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
         }
         if (lane < G) Abuf[(t % kDecNPB) * G + lane] = a;
         kept_mask |= 1ull << (t & 63);
-        if (tid == 0) issue_v(t);
+        if (tid == 0 && !*abort_flag) issue_v(t);
       } else {
         kept_mask &= ~(1ull << (t & 63));
         n_skipped += 1;
@@ -333,11 +329,9 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
     if (u >= 0 && ((kept_mask >> (u & 63)) & 1)) {
       // ---- O = alpha O + P_u V_u over this warp's 8 keys.
       const int vs = u % kDecNV;
-      bad = !__all_sync(0xffffffffu, mbar_wait(vfull(vs), (v_phase >> vs) & 1, abort_flag));
+      mbar_wait(vfull(vs), (v_phase >> vs) & 1, abort_flag);
       v_phase ^= 1u << vs;
-    }
-    if (u >= 0 && ((kept_mask >> (u & 63)) & 1) && !bad) {
-      const int vs = u % kDecNV;
+      __syncwarp();
       const int keys = tile_keys(u);
       const float* Pu = Pbuf + (u % kDecNPB) * kDecKeysPerWarp * G;
       const uint8_t* vtile = smem + L::kV + vs * L::kTileBytes;
@@ -379,14 +373,16 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
     }
   }
 
-  // A wait that gave up in the last tiles' P.V has met no barrier yet.
-  if (!aborted && __syncthreads_or(bad)) aborted = true;
-  if (aborted) {
-    // The split's result is unusable (the status word says why): publish an
-    // empty split, then wait out every copy still in flight before exiting.
-    for (int i = tid; i < G * D; i += kDecThreads)
-      p.o_part[((head0 + i / D) * p.S + split) * D + (i % D)] = 0.f;
-    if (tid < G) p.lse_part[(head0 + tid) * p.S + split] = -INFINITY;
+  // ---- epilogue: merge the warps' partial O and row sums, write the split.
+  // A lane's row-sum share counts once per (key group, head).
+  float lw = owner ? l_lane : 0.f;
+  lw += __shfl_xor_sync(0xffffffffu, lw, 8);
+  lw += __shfl_xor_sync(0xffffffffu, lw, 16);
+  __syncthreads();  // every warp is past its last use of the K ring (and its last wait)
+  if (*abort_flag) {
+    // Every wait is over, so the flag is final here.  Wait out each ring
+    // slot's last copy (those a timed-out wait did not see land) before the
+    // CTA exits and its shared memory is reused.
     if (tid == 0) {
       int no_abort = 0;
 #pragma unroll
@@ -401,13 +397,6 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
     }
     return;
   }
-
-  // ---- epilogue: merge the warps' partial O and row sums, write the split.
-  // A lane's row-sum share counts once per (key group, head).
-  float lw = owner ? l_lane : 0.f;
-  lw += __shfl_xor_sync(0xffffffffu, lw, 8);
-  lw += __shfl_xor_sync(0xffffffffu, lw, 16);
-  __syncthreads();  // every warp is past its last use of the K ring
   float* red = reinterpret_cast<float*>(smem + L::kK);
 #pragma unroll
   for (int g = 0; g < G; ++g)
