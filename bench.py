@@ -1,35 +1,41 @@
 #!/usr/bin/env python
 """Benchmark of Skip-Softmax tiled attention on B200.
 
-One step = one pass of the whole hot path over one batch of synthetic input:
-  * prefill on the Llama-3.1-8B-shaped workload (B=1, Hq=32, Hkv=8, L=16384,
-    d=128, causal, Br=Bc=128, threshold_scale_factor=1000), literal generator
-    reading (|u| = 1, as the workload is written) -- the headline -- and the
-    rms reading (|u| = sqrt(d)) where planted tiles dominate;
+One step = one pass of the whole hot path over one batch of synthetic input of
+every workload (each leg its own kernel launch, L2 flushed before it):
+  * prefill on the Llama-3.3-70B-layer-shaped long workload (B=1, Hq=64,
+    Hkv=8, L=131072, d=128, causal, Br=Bc=128, threshold_scale_factor=1000),
+    literal generator reading (|u| = 1, as the workload is written) -- the
+    headline -- and the rms reading (|u| = sqrt(d)) where planted tiles
+    dominate;
+  * prefill on the Llama-3.1-8B-shaped 16K workload (both readings, also with
+    the per-warp 32-row vote), the video-DiT-shaped non-causal d=64 workload
+    and the tiny 1K workload;
   * split-KV decode on the batch-64 GQA workload (Hq=32, Hkv=8, d=128, KV
     lengths uniform in [16K, 32K], Bc=64, 16 splits, tsf=500) followed by the
-    log-sum-exp merge.
+    log-sum-exp merge, both readings.
 
-The prefill legs also run with the per-warp (32-row slice) vote.
+Every leg is also timed with skipping disabled (factor 0, same kernel) and
+carries its CPU-oracle figure on a sample of whole query tiles.
 
-`value` is the prefill throughput in executed TFLOP/s (tensor work actually
-issued: 2 Br Bc d per visited tile for Q K^T plus 2 Br Bc d per kept tile for
-P V), over all ranks. Dense-equivalent TFLOP/s, skip fractions and the decode
-GB/s on bytes actually moved are reported beside it. `e2e` is the same metric
-through the library's host-memory calls (sskip_attn_prefill_host, which
-overlaps the copies with the kernels, and sskip_attn_decode_host), pinned
-host inputs in and outputs out inside the timed region.
+`value` is the headline prefill throughput in executed TFLOP/s (tensor work
+actually issued: 2 Br Bc d per visited tile for Q K^T plus 2 Br Bc d per kept
+tile for P V), over all ranks. Dense-equivalent TFLOP/s, skip fractions and
+the decode GB/s on bytes actually moved are reported beside it. `e2e` is the
+same metric through the library's host-memory calls (sskip_attn_prefill_host,
+which overlaps the copies with the kernels, and sskip_attn_decode_host),
+pinned host inputs in and outputs out inside the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-Other modes (one GPU): --sweep (speed vs skip over threshold factors),
---calibrate (factors calibrated to target skip ratios), --reorder (video
-workload in raster vs Hilbert token order), --step (one serving step with a
-factor per phase, eager and CUDA-graph replay).
+Other modes (one GPU): --sweep (speed vs skip over threshold factors on the
+128K workload), --calibrate (factors calibrated to target skip ratios),
+--reorder (video workload in raster vs Hilbert token order), --step (one
+serving step with a factor per phase, eager and CUDA-graph replay).
 
 For N > 1 launch under torch.distributed.run: every rank runs an independent
 replica (the method has no cross-GPU exchange), times are maxed over ranks.
-`--impl reference` times the CPU oracle on a bounded sample of the same
+`--impl reference` times the CPU oracle on a bounded sample of the headline
 workload on this host's cores.
 """
 from __future__ import annotations
@@ -205,6 +211,21 @@ def oracle_sample_units(w, heads: int, stride: int = 1) -> np.ndarray:
     return np.array([(0, h, i) for h in range(heads) for i in range(0, w.n_q, stride)], np.int32)
 
 
+def oracle_spread_units(w, n: int) -> np.ndarray:
+    """n whole query tiles of query head 0 spread evenly over the query axis
+    (for a causal workload: over the diagonal, light and heavy tiles alike)."""
+    i = np.unique(np.linspace(0, w.n_q - 1, min(n, w.n_q)).round().astype(int))
+    return np.array([(0, 0, int(t)) for t in i], np.int32)
+
+
+# Short leg names of the prefill workloads.
+SHORT = {synth.LLAMA70B_PREFILL_128K.name: "128k", synth.LLAMA8B_PREFILL_16K.name: "16k",
+         synth.VIDEO_DIT_PREFILL.name: "video", synth.TINY_PREFILL.name: "tiny"}
+
+# Whole query tiles per leg for the CPU-oracle figure (a few seconds each).
+ORACLE_SAMPLE_TILES = {"128k": 8, "16k": 32, "video": 16, "tiny": 16}
+
+
 def time_oracle(w, x, units: np.ndarray, nthreads: int) -> dict:
     import oracle  # CPU oracle: the baseline leg only
     t0 = time.perf_counter()
@@ -218,12 +239,13 @@ def time_oracle(w, x, units: np.ndarray, nthreads: int) -> dict:
 
 def run_reference(args, w, rank: int):
     """CPU oracle as the reference arm: each step is a bounded sample of the
-    workload (a stratified quarter of one query head's tiles)."""
+    workload (32 whole query tiles of one query head, spread over the query
+    axis)."""
     if rank != 0:
         return
     x = synth.prefill_inputs(w, args.reading)
     threads = os.cpu_count() or 1
-    step_units = oracle_sample_units(w, heads=1, stride=4)
+    step_units = oracle_spread_units(w, 32)
     for _ in range(args.warmup):
         time_oracle(w, x, step_units, threads)
     secs, flops = 0.0, 0.0
@@ -232,8 +254,8 @@ def run_reference(args, w, rank: int):
         secs += r["seconds"]
         flops += r["executed_flops"]
     value = flops / secs / 1e12
-    sample = (f"per step {len(step_units)} whole 128-row query tiles (every 4th tile of query "
-              f"head 0) of {w.name}, {args.reading} reading")
+    sample = (f"per step {len(step_units)} whole {w.Br}-row query tiles of query head 0 spread "
+              f"evenly over the query axis, of {w.name}, {args.reading} reading")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -250,7 +272,10 @@ def config_block(w, args) -> dict:
     dw = decode_workload(args)
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "d": w.d,
             "causal": w.causal, "Br": w.Br, "Bc": w.Bc, "threshold_scale_factor": w.tsf,
-            "generator_reading": args.reading, "decode_workload": dw.name,
+            "generator_reading": args.reading,
+            "other_prefill_workloads": [n for n in args.extra_prefill.split(",")
+                                        if n and n != w.name],
+            "decode_workload": dw.name,
             "decode_threshold_scale_factor": dw.tsf, "decode_num_splits": dw.num_splits,
             "l2": "flushed before every timed kernel (256 MiB write)",
             "only": args.only, "parallelism": f"replicas x{args.gpus}"}
@@ -288,39 +313,49 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
     warp_readings = [r for r in args.warp_vote_readings.split(",") if r]
     dw = decode_workload(args)
 
-    # ---- legs of the step: prefill and decode, one per generator reading.
+    # ---- legs of the step: every prefill workload per generator reading,
+    # then decode. The video workload has one reading (its generator has no
+    # planted direction).
+    works = [w] + [synth.PREFILL_WORKLOADS[n] for n in args.extra_prefill.split(",")
+                   if n and n != w.name]
     legs = []
     if args.only != "decode":
-        for rd in readings:
-            x = synth.prefill_inputs(w, rd)
-            t = {"q": to_dev(x["q"]), "k": to_dev(x["k"]), "v": to_dev(x["v"])}
-            t["o"] = torch.empty_like(t["q"])
-            t["lse"] = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
-            t["cnt"] = torch.zeros(2, dtype=torch.int64, device=dev)
+        for wk in works:
+            short = SHORT[wk.name]
+            for rd in (["lit"] if wk.kind == "video" else readings):
+                x = synth.prefill_inputs(wk, rd)
+                t = {"q": to_dev(x["q"]), "k": to_dev(x["k"]), "v": to_dev(x["v"])}
+                t["o"] = torch.empty_like(t["q"])
+                t["lse"] = torch.empty((wk.B, wk.Hq, wk.L), dtype=torch.float32, device=dev)
+                t["cnt"] = torch.zeros(2, dtype=torch.int64, device=dev)
 
-            def run(t=t, tsf=None, tiles=None):
-                sk.sskip_attn_prefill(t["q"], t["k"], t["v"], t["o"], t["lse"], causal=w.causal,
-                                      sm_scale=w.scale,
-                                      threshold_scale_factor=w.tsf if tsf is None else tsf,
-                                      Br=w.Br, Bc=w.Bc, skip_count=t["cnt"], tile_state=tiles,
-                                      stream=stream)
-            legs.append({"name": f"prefill_{rd}", "kind": "prefill", "reading": rd, "t": t,
-                         "host": x, "run": run, "launches": 1, "w": w})
-            if rd in warp_readings:
-                # Same inputs, vote taken per 32-row warp slice.
-                tw = dict(t, o=torch.empty_like(t["q"]),
-                          lse=torch.empty_like(t["lse"]),
-                          cnt=torch.zeros(4, dtype=torch.int64, device=dev))
+                def run(t=t, wk=wk, tsf=None, tiles=None):
+                    sk.sskip_attn_prefill(t["q"], t["k"], t["v"], t["o"], t["lse"],
+                                          causal=wk.causal, sm_scale=wk.scale,
+                                          threshold_scale_factor=wk.tsf if tsf is None else tsf,
+                                          Br=wk.Br, Bc=wk.Bc, skip_count=t["cnt"],
+                                          tile_state=tiles, stream=stream)
+                head = wk is w and rd == args.reading
+                legs.append({"name": f"prefill_{short}_{rd}", "key": f"{short}_{rd}",
+                             "kind": "prefill", "reading": rd, "t": t, "host": x, "run": run,
+                             "launches": 1, "w": wk, "headline": head, "e2e": head})
+                if wk.name == args.warp_vote_workload and rd in warp_readings:
+                    # Same inputs, vote taken per 32-row warp slice.
+                    tw = dict(t, o=torch.empty_like(t["q"]), lse=torch.empty_like(t["lse"]),
+                              cnt=torch.zeros(4, dtype=torch.int64, device=dev))
 
-                def run_w(t=tw, tsf=None, tiles=None):
-                    sk.sskip_attn_prefill_vote(
-                        t["q"], t["k"], t["v"], t["o"], t["lse"], causal=w.causal,
-                        sm_scale=w.scale, threshold_scale_factor=w.tsf if tsf is None else tsf,
-                        Br=w.Br, Bc=w.Bc, vote_rows=32, counts=t["cnt"], tile_state=tiles,
-                        stream=stream)
-                legs.append({"name": f"prefill_{rd}_warp32", "kind": "prefill", "reading": rd,
-                             "vote": "warp32", "t": tw, "host": x, "run": run_w, "launches": 1,
-                             "extra": True})
+                    def run_w(t=tw, wk=wk, tsf=None, tiles=None):
+                        sk.sskip_attn_prefill_vote(
+                            t["q"], t["k"], t["v"], t["o"], t["lse"], causal=wk.causal,
+                            sm_scale=wk.scale,
+                            threshold_scale_factor=wk.tsf if tsf is None else tsf,
+                            Br=wk.Br, Bc=wk.Bc, vote_rows=32, counts=t["cnt"], tile_state=tiles,
+                            stream=stream)
+                    legs.append({"name": f"prefill_{short}_{rd}_warp32",
+                                 "key": f"{short}_{rd}_warp32", "kind": "prefill",
+                                 "reading": rd, "vote": "warp32", "block_leg": f"prefill_{short}_{rd}",
+                                 "t": tw, "host": x, "run": run_w, "launches": 1, "w": wk,
+                                 "extra": True})
     if args.only != "prefill":
         for rd in (readings if args.decode_readings == "all" else [args.reading]):
             dx = synth.decode_inputs(dw, rd)
@@ -339,19 +374,21 @@ def run_gpu(args, w, rank: int, world: int, local_rank: int):
                                      threshold_scale_factor=dw.tsf if tsf is None else tsf,
                                      Bc=dw.Bc, num_splits=dw.num_splits, workspace=t["ws"],
                                      skip_count=t["cnt"], tile_state=tiles, stream=stream)
-            legs.append({"name": f"decode_{rd}", "kind": "decode", "reading": rd, "t": t,
-                         "host": {"q": dx["q"], "seqlens": dx["seqlens"]}, "run": run,
-                         "launches": 2, "dw": dw})
+            legs.append({"name": f"decode_{rd}", "key": rd, "kind": "decode", "reading": rd,
+                         "t": t, "host": {"q": dx["q"], "seqlens": dx["seqlens"]}, "run": run,
+                         "launches": 2, "dw": dw, "e2e": rd == args.reading})
             del dx
 
     # ---- one untimed pass with tile records: skip counts, FLOPs, bytes moved
     for leg in legs:
         t = leg["t"]
         if leg["kind"] == "prefill":
-            tiles = torch.empty((w.B, w.Hq, w.n_q, w.n_k), dtype=torch.uint8, device=dev)
+            wk = leg["w"]
+            tiles = torch.empty((wk.B, wk.Hq, wk.n_q, wk.n_k), dtype=torch.uint8, device=dev)
             leg["run"](tiles=tiles)
             c = t["cnt"].cpu().tolist()
-            leg["stats"] = {"skipped": c[0], "visited": c[1], **prefill_flops(w, c[1], c[0])}
+            leg["stats"] = {"skipped": c[0], "visited": c[1], **prefill_flops(wk, c[1], c[0])}
+            del tiles
             if len(c) == 4:
                 leg["stats"].update(slices_skipped=c[2], slices_visited=c[3])
         else:
@@ -423,7 +460,7 @@ def time_e2e(legs, flush, stream, new_events, timed, steps, kv_per_chunk=0):
     """Same steps with each leg's inputs copied host->device from pinned memory
     and its outputs copied back inside the timed region."""
     import torch
-    legs = [leg for leg in legs if not leg.get("extra")]
+    legs = [leg for leg in legs if leg.get("e2e")]
     h2d = d2h = 0
     for leg in legs:
         t = leg["t"]
@@ -471,6 +508,19 @@ def time_e2e(legs, flush, stream, new_events, timed, steps, kv_per_chunk=0):
     return timed(e2e_step, steps, only=[leg["name"] for leg in legs]), (h2d, d2h)
 
 
+def leg_oracle_baseline(leg) -> dict:
+    """The CPU oracle on a sample of whole query tiles of the leg's inputs."""
+    wk = leg["w"]
+    units = oracle_spread_units(wk, ORACLE_SAMPLE_TILES[SHORT[wk.name]])
+    threads = os.cpu_count() or 1
+    r = time_oracle(wk, leg["host"], units, threads)
+    return {"value": r["executed_flops"] / r["seconds"] / 1e12, "unit": "TFLOP/s",
+            "cores": threads, "kind": "oracle", "seconds": r["seconds"],
+            "sample": (f"{len(units)} whole {wk.Br}-row query tiles of query head 0 spread "
+                       f"evenly over the query axis, {wk.name}, {leg['reading']} reading; "
+                       f"executed FLOPs / wall time")}
+
+
 def report(args, w, dw, world, legs, ms, ms_dense, ems, io_bytes, peaks, peak_kind,
            clock_rec) -> dict:
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -481,13 +531,15 @@ def report(args, w, dw, world, legs, ms, ms_dense, ems, io_bytes, peaks, peak_ki
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_block(w, args)}
     pre, dec = {}, {}
+    cpu_ok = not args.no_cpu_baseline and world == 1
     for leg in legs:
         n, s = leg["name"], leg["stats"]
         t = ms[n] / 1e3
         b = {"ms_per_launch": ms[n], "skip_fraction": s["skipped"] / max(1, s["visited"]),
              "skipped_tiles": s["skipped"], "visited_tiles": s["visited"]}
         if leg["kind"] == "prefill":
-            b.update(executed_tflops=s["executed"] / t / 1e12,
+            b.update(workload=leg["w"].name, reading=leg["reading"],
+                     executed_tflops=s["executed"] / t / 1e12,
                      dense_equiv_tflops=s["dense"] / t / 1e12,
                      executed_frac_of_peak=s["executed"] / t / 1e12 / peak,
                      executed_tflop=s["executed"] / 1e12, dense_equiv_tflop=s["dense"] / 1e12)
@@ -502,33 +554,38 @@ def report(args, w, dw, world, legs, ms, ms_dense, ems, io_bytes, peaks, peak_ki
                      ideal_speedup=ideal)
         if n in ems:
             b["e2e_ms"] = ems[n]
-        key = leg["reading"]
         if leg.get("vote"):
-            key = f"{key}_{leg['vote']}"
             b.update(vote_rows=32, slice_skip_fraction=s["slices_skipped"] / max(1, s["slices_visited"]),
                      slices_skipped=s["slices_skipped"], slices_visited=s["slices_visited"])
-            blk = f"prefill_{leg['reading']}"
-            if blk in ms:
-                b["speedup_vs_block_vote"] = ms[blk] / ms[n]
-        (pre if leg["kind"] == "prefill" else dec)[key] = b
-    head = args.reading
-    if pre:
-        hs = next(leg["stats"] for leg in legs if leg["name"] == f"prefill_{head}")
-        t = ms[f"prefill_{head}"] / 1e3
+            if leg["block_leg"] in ms:
+                b["speedup_vs_block_vote"] = ms[leg["block_leg"]] / ms[n]
+        elif leg["kind"] == "prefill" and cpu_ok:
+            b["cpu_baseline"] = leg_oracle_baseline(leg)
+        (pre if leg["kind"] == "prefill" else dec)[leg["key"]] = b
+    head = next((leg for leg in legs if leg.get("headline")), None)
+    if head is not None:
+        hs = head["stats"]
+        t = ms[head["name"]] / 1e3
         achieved = hs["executed"] / t / 1e12
         line["value"] = world * achieved
         line["roofline"] = {
             "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": ncu_traffic("prefill_kernel"),
             "kernel": f"prefill_kernel<{w.d},{w.Br},{w.Bc},{'causal' if w.causal else 'full'}>",
-            "peak_source": f"{peak_kind} bf16_tflops (burst; kernel timed alone)"}
+            "leg": head["key"],
+            "peak_source": f"{peak_kind} bf16_tflops (burst; the SM clock stays at its maximum "
+                           f"during the step)"}
         line["prefill"] = pre
-        if ems:
-            line["e2e"] = {"value": world * hs["executed"] / (ems[f"prefill_{head}"] / 1e3) / 1e12,
+        if head["name"] in ems:
+            line["e2e"] = {"value": world * hs["executed"] / (ems[head["name"]] / 1e3) / 1e12,
                            "unit": "TFLOP/s", "h2d_bytes_per_step": io_bytes[0],
-                           "d2h_bytes_per_step": io_bytes[1]}
+                           "d2h_bytes_per_step": io_bytes[1], "leg": head["key"]}
+        if "cpu_baseline" in pre[head["key"]]:
+            line["cpu_baseline"] = pre[head["key"]]["cpu_baseline"]
+    elif pre:
+        line["prefill"] = pre
     if dec:
-        dkey = head if head in dec else next(iter(dec))
+        dkey = args.reading if args.reading in dec else next(iter(dec))
         dstats = next(leg["stats"] for leg in legs if leg["name"] == f"decode_{dkey}")
         gbs = dec[dkey]["gbs_actually_moved"]
         dec["workload"] = dw.name
@@ -536,25 +593,14 @@ def report(args, w, dw, world, legs, ms, ms_dense, ems, io_bytes, peaks, peak_ki
                            "frac": gbs / hbm, "traffic": ncu_traffic("decode_split_kernel"),
                            "reading": dkey, "peak_source": f"{peak_kind} hbm_gbs"}
         line["decode"] = dec
-        if not pre:  # decode-only runs report GB/s as the value
+        if head is None:  # decode-only runs report GB/s as the value
             line.update(value=world * gbs, unit="GB/s", roofline=dec["roofline"])
-            if ems:
+            if f"decode_{dkey}" in ems:
                 line["e2e"] = {"value": world * dstats["total"] / (ems[f"decode_{dkey}"] / 1e3) / 1e9,
                                "unit": "GB/s", "h2d_bytes_per_step": io_bytes[0],
                                "d2h_bytes_per_step": io_bytes[1]}
     line["clocks"] = clock_rec
     line["gpu_launches"] = sum(leg["launches"] for leg in legs) * K
-    if not args.no_cpu_baseline and world == 1 and pre:
-        units = oracle_sample_units(w, heads=args.cpu_heads)
-        threads = os.cpu_count() or 1
-        hx = next(leg["host"] for leg in legs if leg["name"] == f"prefill_{head}")
-        r = time_oracle(w, hx, units, threads)
-        line["cpu_baseline"] = {
-            "value": r["executed_flops"] / r["seconds"] / 1e12, "unit": "TFLOP/s",
-            "cores": threads, "kind": "oracle", "seconds": r["seconds"],
-            "sample": (f"all {w.n_q} query tiles of {args.cpu_heads} of {w.Hq} query heads "
-                       f"({args.cpu_heads / w.Hq:.3f} of {w.name}, {head} reading), "
-                       f"executed FLOPs / wall time")}
     return line
 
 
@@ -738,8 +784,7 @@ def run_reorder(args):
     peaks, _ = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    w = synth.VIDEO_DIT_PREFILL if args.prefill == synth.LLAMA8B_PREFILL_16K.name \
-        else synth.PREFILL_WORKLOADS[args.prefill]
+    w = synth.PREFILL_WORKLOADS[args.prefill]
     if args.tsf is not None:
         w = w.replace(tsf=args.tsf)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
@@ -892,8 +937,15 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--prefill", default=synth.LLAMA8B_PREFILL_16K.name,
-                    choices=sorted(synth.PREFILL_WORKLOADS))
+    ap.add_argument("--prefill", default=None, choices=sorted(synth.PREFILL_WORKLOADS),
+                    help="headline prefill workload (default: the 128K workload; --calibrate "
+                         "and --step default to the 16K one, --reorder to the video one)")
+    ap.add_argument("--extra-prefill", default=",".join(
+                        n.name for n in (synth.LLAMA8B_PREFILL_16K, synth.VIDEO_DIT_PREFILL,
+                                         synth.TINY_PREFILL)),
+                    help="further prefill workloads timed as legs of the step ('' for none)")
+    ap.add_argument("--warp-vote-workload", default=synth.LLAMA8B_PREFILL_16K.name,
+                    help="the workload whose legs are also timed with the per-warp vote")
     ap.add_argument("--decode", default=synth.DECODE_B64_32K.name,
                     choices=sorted(synth.DECODE_WORKLOADS))
     ap.add_argument("--tsf", type=float, default=None, help="override the prefill factor")
@@ -903,7 +955,6 @@ def main(argv=None):
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="restrict the step (profiling of one kernel on a small device footprint)")
     ap.add_argument("--decode-batch", type=int, default=0, help="override the decode batch")
-    ap.add_argument("--cpu-heads", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-kv-per-chunk", type=int, default=0,
@@ -927,6 +978,10 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
+    if args.prefill is None:
+        args.prefill = (synth.LLAMA8B_PREFILL_16K.name if (args.calibrate or args.step) else
+                        synth.VIDEO_DIT_PREFILL.name if args.reorder else
+                        synth.LLAMA70B_PREFILL_128K.name)
     w = synth.PREFILL_WORKLOADS[args.prefill]
     if args.tsf is not None:
         w = w.replace(tsf=args.tsf)

@@ -94,3 +94,48 @@ def test_reference_arm_under_torchrun_prints_on_rank0_only():
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1 and json.loads(lines[0])["n_gpus"] == 2
+
+
+def test_spread_units_and_leg_names():
+    w = synth.LLAMA70B_PREFILL_128K
+    u = bench.oracle_spread_units(w, 32)
+    assert len(u) == 32 and u[0].tolist() == [0, 0, 0] and u[-1].tolist() == [0, 0, w.n_q - 1]
+    assert np.all(np.diff(u[:, 2]) > 0)
+    tiny = bench.oracle_spread_units(synth.TINY_PREFILL, 100)
+    assert len(tiny) == synth.TINY_PREFILL.n_q  # never more tiles than the workload has
+    assert set(bench.SHORT) == set(synth.PREFILL_WORKLOADS)
+    assert set(bench.ORACLE_SAMPLE_TILES) == set(bench.SHORT.values())
+
+
+def test_report_headline_and_legs():
+    """report() on made-up leg timings: the headline value, roofline and
+    per-leg fields come from the headline leg's executed FLOPs and time."""
+    args = bench.main.__globals__["argparse"].Namespace(
+        steps=10, warmup=3, gpus=1, reading="lit", only="all", no_cpu_baseline=True,
+        extra_prefill=synth.LLAMA8B_PREFILL_16K.name, decode=synth.DECODE_B64_32K.name,
+        decode_batch=0)
+    w, w16 = synth.LLAMA70B_PREFILL_128K, synth.LLAMA8B_PREFILL_16K
+    dw = synth.DECODE_B64_32K
+    n = w.n_q
+    vis = w.Hq * n * (n + 1) // 2
+    legs = [
+        {"name": "prefill_128k_lit", "key": "128k_lit", "kind": "prefill", "reading": "lit",
+         "w": w, "launches": 1, "headline": True,
+         "stats": {"skipped": 0, "visited": vis, **bench.prefill_flops(w, vis, 0)}},
+        {"name": "prefill_16k_rms", "key": "16k_rms", "kind": "prefill", "reading": "rms",
+         "w": w16, "launches": 1,
+         "stats": {"skipped": 50, "visited": 100, **bench.prefill_flops(w16, 100, 50)}},
+    ]
+    ms = {"prefill_128k_lit": 280.0, "prefill_16k_rms": 1.0}
+    ms_dense = {"prefill_128k_lit": 280.0, "prefill_16k_rms": 1.5}
+    peaks = {"bf16_tflops": 1600.0, "hbm_gbs": 6400.0}
+    line = bench.report(args, w, dw, 1, legs, ms, ms_dense, {}, (0, 0), peaks, "measured",
+                        {"sm_mhz": 1965})
+    ex = 2.0 * 128 * 128 * 128 * 2 * vis
+    assert line["value"] == pytest.approx(ex / 0.280 / 1e12)
+    assert line["roofline"]["frac"] == pytest.approx(line["value"] / 1600.0)
+    assert line["roofline"]["leg"] == "128k_lit" and line["config"]["workload"] == w.name
+    p = line["prefill"]["16k_rms"]
+    assert p["skip_fraction"] == 0.5 and p["speedup_vs_skip_disabled"] == pytest.approx(1.5)
+    assert p["ideal_speedup"] == pytest.approx(1 / 0.75)
+    assert line["gpu_launches"] == 2 * 10
