@@ -83,8 +83,8 @@ constexpr int kPfVoteSlots = 4;
 #ifndef SSKIP_PF_NACC
 #define SSKIP_PF_NACC 4       // independent packed accumulators of the row sum
 #endif
-#ifndef SSKIP_PF_SPLIT_S
-#define SSKIP_PF_SPLIT_S 0    // S(j+1) as two halves, the upper one issued before P(j) is done
+#ifndef SSKIP_PF_TRIPLE
+#define SSKIP_PF_TRIPLE 1     // three rotating S buffers where TMEM has room (3 Bc + 2 d <= 512)
 #endif
 #ifndef SSKIP_PF_ROUNDED_L
 #define SSKIP_PF_ROUNDED_L 0  // 1: O is divided by the sum of the bf16 P that P.V used
@@ -123,17 +123,22 @@ struct PrefillCfg {
   static constexpr int kK = kQ + 2 * kQBytes;
   static constexpr int kV = kK + kNK * kKVBytes;
   static constexpr int kBar = kV + kNV * kKVBytes;
+  // Three S/P buffers that rotate over the two query tiles' key tiles when
+  // TMEM holds them next to the two O accumulators; else one per query tile.
+  static constexpr bool kTriple = SSKIP_PF_TRIPLE != 0 && 3 * BC + 2 * D <= 512;
+  static constexpr int kSBufs = kTriple ? 3 : 2;
+  static constexpr int kOCol = kSBufs * BC;  // first TMEM column of O_A (O_B follows)
   // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], then per
-  // warpgroup s_full, vote_mma, p_lo, s_hi_free, p_hi, then
+  // warpgroup s_full[2], vote_mma[2], p_lo[2], p_hi[2], o_done, then
   // vote_full[2][VS], vote_empty[2][VS], mma_done
-  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 5 * 2 + 4 * kPfVoteSlots + 1;
+  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 9 * 2 + 4 * kPfVoteSlots + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   // kept flags [2 wg][2 parity], vote_kept[VS][2], warp vote flags
   // [2 wg][2 parity][4], tmem, abort, warp gaps [2 wg][2 parity][4] (fp32)
   static constexpr int kMiscInts = 4 + 2 * kPfVoteSlots + 16 + 2 + 16;
   static constexpr int kTotal = kMisc + kMiscInts * 4;
   static constexpr int kAlloc = kTotal + 1024;  // room to align the base to 1 KB
-  static constexpr int kTmemCols = (2 * BC + 2 * D) <= 256 ? 256 : 512;
+  static constexpr int kTmemCols = (kOCol + 2 * D) <= 256 ? 256 : 512;
   static_assert(kQBytes % 1024 == 0 && kKVBytes % 1024 == 0, "tiles keep 1 KB alignment");
   static_assert(kAlloc <= 227 * 1024, "shared memory budget");
 };
@@ -166,9 +171,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   constexpr int WPG = BR / 32;    // warps per vote group
   constexpr int HK = BC / 2;      // keys per half tile
   constexpr int HP = HK / 2;      // packed bf16 P columns per half tile
-  constexpr bool SPLIT = SSKIP_PF_SPLIT_S != 0;
+  constexpr bool TRIPLE = C::kTriple;
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BC, 0, 0);
-  constexpr uint32_t IDESC_SH = idesc_bf16_f32(128, HK, 0, 0);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
   static_assert(BR == 64 || BR == 128, "Br");
   static_assert(BC == 64 || BC == 128, "Bc");
@@ -191,16 +195,33 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   auto b_vfull = [&](int s) { return smem_u32(&bars[1 + 2 * NK + s]); };
   auto b_vempty = [&](int s) { return smem_u32(&bars[1 + 2 * NK + NV + s]); };
   constexpr int kWgBar = 1 + 2 * NK + 2 * NV;
-  auto b_sfull = [&](int w) { return smem_u32(&bars[kWgBar + w]); };      // MMA -> softmax
-  auto b_vmma = [&](int w) { return smem_u32(&bars[kWgBar + 2 + w]); };  // decision -> MMA
-  auto b_plo = [&](int w) { return smem_u32(&bars[kWgBar + 4 + w]); };   // P_lo stored
-  auto b_hfree = [&](int w) { return smem_u32(&bars[kWgBar + 6 + w]); }; // upper S re-read
-  auto b_phi = [&](int w) { return smem_u32(&bars[kWgBar + 8 + w]); };   // P_hi stored
-  auto b_vote_full = [&](int w, int s) { return smem_u32(&bars[kWgBar + 10 + w * VS + s]); };
-  auto b_vote_empty = [&](int w, int s) {
-    return smem_u32(&bars[kWgBar + 10 + 2 * VS + w * VS + s]);
+  // Signals between a query tile's softmax and the MMA thread, each in two
+  // barriers taken by the parity of its index (key tile j, or kept tile k):
+  // with three S buffers a softmax step may run one tile ahead of the MMA
+  // thread's handling of the previous one, and one barrier could then
+  // complete two phases before the other side tests the first.
+  //   s_full  S(w, j) is in TMEM                 (MMA -> softmax)
+  //   vote    the decision on tile j is posted   (softmax -> MMA)
+  //   p_lo    P of the first Bc/2 keys stored    (softmax -> MMA, kept tiles)
+  //   p_hi    all of P stored                    (softmax -> MMA, kept tiles)
+  // (With one S buffer per query tile neither side can run ahead, so the
+  // first barrier of each pair serves every index.)
+  auto b_pair = [&](int base, int w, int i) {
+    return smem_u32(&bars[kWgBar + base + 2 * w + (TRIPLE ? (i & 1) : 0)]);
   };
-  const uint32_t b_mmadone = smem_u32(&bars[kWgBar + 10 + 4 * VS]);
+  auto pair_par = [&](int i) { return uint32_t(TRIPLE ? (i >> 1) & 1 : i & 1); };
+  auto b_sfull = [&](int w, int j) { return b_pair(0, w, j); };
+  auto b_vmma = [&](int w, int j) { return b_pair(4, w, j); };
+  auto b_plo = [&](int w, int k) { return b_pair(8, w, k); };
+  auto b_phi = [&](int w, int k) { return b_pair(12, w, k); };
+  auto b_odone = [&](int w) { return smem_u32(&bars[kWgBar + 16 + w]); }; // P.V of a kept tile done
+  auto b_vote_full = [&](int w, int s) { return smem_u32(&bars[kWgBar + 18 + w * VS + s]); };
+  auto b_vote_empty = [&](int w, int s) {
+    return smem_u32(&bars[kWgBar + 18 + 2 * VS + w * VS + s]);
+  };
+  const uint32_t b_mmadone = smem_u32(&bars[kWgBar + 18 + 4 * VS]);
+  // TMEM column of the S/P buffer of query tile w at key tile j.
+  auto s_col = [&](int w, int j) { return uint32_t((TRIPLE ? (2 * j + w) % 3 : w) * BC); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -233,11 +254,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int s = 0; s < NK; ++s) { mbar_init(b_kfull(s), 1); mbar_init(b_kempty(s), 1); }
     for (int s = 0; s < NV; ++s) { mbar_init(b_vfull(s), 1); mbar_init(b_vempty(s), 1); }
     for (int w = 0; w < 2; ++w) {
-      mbar_init(b_sfull(w), 1);
-      mbar_init(b_vmma(w), 1);
-      mbar_init(b_plo(w), 4);    // one arrival per softmax warp
-      mbar_init(b_hfree(w), 4);
-      mbar_init(b_phi(w), 4);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(b_sfull(w, i), 1);
+        mbar_init(b_vmma(w, i), 1);
+        mbar_init(b_plo(w, i), 4);  // one arrival per softmax warp
+        mbar_init(b_phi(w, i), 4);
+      }
+      mbar_init(b_odone(w), 1);
     }
     for (int w = 0; w < 2; ++w)
       for (int s = 0; s < VS; ++s) { mbar_init(b_vote_full(w, s), 1); mbar_init(b_vote_empty(w, s), 1); }
@@ -292,24 +315,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint64_t dq0 = smem_desc_sw128(sbase + C::kQ, 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(sbase + C::kK, 16, 1024);
       const uint64_t dv0 = smem_desc_sw128(sbase + C::kV, BC * 128, 1024);
-      // Keys [k0, k0 + n) of S(w, j), n = Bc or Bc / 2, from key rows
-      // [k0, k0 + n) of the K tile (whole 1 KB swizzle atoms).
-      auto issue_s = [&](int w, int j, int k0, uint32_t idesc) {
+      // S = Q_w K_j^T into TMEM columns [col, col + Bc).
+      auto issue_s = [&](int w, int j, uint32_t col) {
         const uint64_t da = dq0 + (uint64_t)((w * C::kQBytes) >> 4);
-        const uint64_t db = dk0 + (uint64_t)(((j % NK) * C::kKVBytes + k0 * 128) >> 4);
-        const uint32_t d_tmem = tmem + w * BC + k0;
+        const uint64_t db = dk0 + (uint64_t)(((j % NK) * C::kKVBytes) >> 4);
+        const uint32_t d_tmem = tmem + col;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oa = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
           const uint32_t ob = ((kk >> 2) * (BC * 128) + (kk & 3) * 32) >> 4;
-          umma_ss(d_tmem, da + oa, db + ob, idesc, kk > 0 ? 1u : 0u);
+          umma_ss(d_tmem, da + oa, db + ob, IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
       int pv_count[2] = {0, 0};
-      // O(w) += P(w)[:, half h] V[half h] from V slot vs; P read from TMEM.
-      auto issue_pv_half = [&](int w, int vs, int h) {
-        const uint32_t p_tmem = tmem + w * BC;
-        const uint32_t o_tmem = tmem + 2 * BC + w * D;
+      // O(w) += P[:, half h] V[half h], P read from TMEM columns from col, V
+      // from slot vs.
+      auto issue_pv_half = [&](int w, uint32_t col, int vs, int h) {
+        const uint32_t p_tmem = tmem + col;
+        const uint32_t o_tmem = tmem + C::kOCol + w * D;
         const uint64_t dv = dv0 + (uint64_t)((vs * C::kKVBytes) >> 4);
 #pragma unroll
         for (int k2 = 0; k2 < HK / 16; ++k2) {
@@ -320,84 +343,129 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (h == 1) ++pv_count[w];
       };
       const int n_w[2] = {n_a, n_b};
-      int kc_w[2] = {0, 0};  // kept tiles per warpgroup: parity of p_lo / s_hi_free / p_hi
+      int kc_w[2] = {0, 0};  // kept tiles per warpgroup: index of p_lo / p_hi / o_done
+      int kc = 0;            // tiles some warpgroup kept: the V load number
       bool ok = mbar_wait(b_qfull, 0, abort_flag);
-      if (ok && n_j > 0) {
-        ok = mbar_wait(b_kfull(0), 0, abort_flag);
-        tc_fence_after();
-        if (ok) {
+      if constexpr (!TRIPLE) {
+        // One S buffer per query tile.  Key tile j, warpgroup A then B: its
+        // decision; for a kept tile P_lo V as soon as P_lo is stored and P_hi V
+        // once P is complete; then S(j+1), which overwrites the P(j) that P.V
+        // just read.  V_j is in slot kc % NV (the V producer's numbering).
+        if (ok && n_j > 0) {
+          ok = mbar_wait(b_kfull(0), 0, abort_flag);
+          tc_fence_after();
+          if (ok) {
 #pragma unroll
-          for (int w = 0; w < 2; ++w)
-            if (n_w[w] > 0) {
-              issue_s(w, 0, 0, IDESC_S);
-              umma_commit(b_sfull(w));
-            }
-          umma_commit(b_kempty(0));
-        }
-      }
-      // Key tile j, warpgroup A then B: the decision; for a kept tile P_lo V
-      // as soon as P_lo is stored and P_hi V once P is complete; then
-      // S(j+1) (with the split option, its upper half as soon as the upper S
-      // columns of tile j have been re-read).  V_j goes to slot (number of
-      // earlier tiles some warpgroup kept) % NV, the V producer's numbering.
-      int kc = 0;
-      for (int j = 0; ok && j < n_j; ++j) {
-        const int vs = kc % NV;
-        const bool nxt = j + 1 < n_j;
-        bool any_kept = false, v_ready = false, k_ready = false;
-        // K_{j+1} is waited for just before its first use, so that a late
-        // K tile never holds back a P.V.
-        auto need_k = [&]() {
-          if (!k_ready) k_ready = mbar_wait(b_kfull((j + 1) % NK), ((j + 1) / NK) & 1, abort_flag);
-          return k_ready;
-        };
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-          if (j >= n_w[w]) continue;
-          const bool s_next = j + 1 < n_w[w];
-          if (!mbar_wait(b_vmma(w), j & 1, abort_flag)) { ok = false; break; }
-          const bool kept = kflag[w * 2 + (j & 1)] != 0;
-          if (kept) {
-            any_kept = true;
-            const uint32_t par = kc_w[w] & 1;
-            if (!mbar_wait(b_plo(w), par, abort_flag)) { ok = false; break; }
-            if (!v_ready) {
-              if (!mbar_wait(b_vfull(vs), (kc / NV) & 1, abort_flag)) { ok = false; break; }
-              v_ready = true;
-            }
-            tc_fence_after();
-            issue_pv_half(w, vs, 0);
-            if (SPLIT && s_next) {
-              if (!mbar_wait(b_hfree(w), par, abort_flag) || !need_k()) { ok = false; break; }
-              tc_fence_after();
-              issue_s(w, j + 1, HK, IDESC_SH);
-            }
-            if (!mbar_wait(b_phi(w), par, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv_half(w, vs, 1);
-            ++kc_w[w];
-            if (s_next) {
-              if (!need_k()) { ok = false; break; }
-              issue_s(w, j + 1, 0, SPLIT ? IDESC_SH : IDESC_S);
-            }
-          } else if (s_next) {
-            if (!need_k()) { ok = false; break; }
-            tc_fence_after();
-            if constexpr (SPLIT) {
-              issue_s(w, j + 1, HK, IDESC_SH);
-              issue_s(w, j + 1, 0, IDESC_SH);
-            } else {
-              issue_s(w, j + 1, 0, IDESC_S);
-            }
+            for (int w = 0; w < 2; ++w)
+              if (n_w[w] > 0) {
+                issue_s(w, 0, w * BC);
+                umma_commit(b_sfull(w, 0));
+              }
+            umma_commit(b_kempty(0));
           }
-          if (s_next) umma_commit(b_sfull(w));
         }
-        if (!ok) break;
-        if (any_kept) {
-          umma_commit(b_vempty(vs));
-          ++kc;
+        for (int j = 0; ok && j < n_j; ++j) {
+          const int vs = kc % NV;
+          bool any_kept = false, v_ready = false, k_ready = false;
+          // K_{j+1} is waited for just before its first use, so that a late
+          // K tile never holds back a P.V.
+          auto need_k = [&]() {
+            if (!k_ready) k_ready = mbar_wait(b_kfull((j + 1) % NK), ((j + 1) / NK) & 1, abort_flag);
+            return k_ready;
+          };
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            if (j >= n_w[w]) continue;
+            const bool s_next = j + 1 < n_w[w];
+            if (!mbar_wait(b_vmma(w, j), pair_par(j), abort_flag)) { ok = false; break; }
+            const bool kept = kflag[w * 2 + (j & 1)] != 0;
+            if (kept) {
+              any_kept = true;
+              const uint32_t par = pair_par(kc_w[w]);
+              if (!mbar_wait(b_plo(w, kc_w[w]), par, abort_flag)) { ok = false; break; }
+              if (!v_ready) {
+                if (!mbar_wait(b_vfull(vs), (kc / NV) & 1, abort_flag)) { ok = false; break; }
+                v_ready = true;
+              }
+              tc_fence_after();
+              issue_pv_half(w, w * BC, vs, 0);
+              if (!mbar_wait(b_phi(w, kc_w[w]), par, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+              issue_pv_half(w, w * BC, vs, 1);
+              ++kc_w[w];
+              if (s_next) {
+                if (!need_k()) { ok = false; break; }
+                issue_s(w, j + 1, w * BC);
+              }
+            } else if (s_next) {
+              if (!need_k()) { ok = false; break; }
+              tc_fence_after();
+              issue_s(w, j + 1, w * BC);
+            }
+            if (s_next) umma_commit(b_sfull(w, j + 1));
+          }
+          if (!ok) break;
+          if (any_kept) {
+            umma_commit(b_vempty(vs));
+            ++kc;
+          }
+          if (j + 1 < n_j) umma_commit(b_kempty((j + 1) % NK));
         }
-        if (nxt) umma_commit(b_kempty((j + 1) % NK));
+      } else {
+        // Three S buffers.  Key tile j: A's tile j, S_B(j+1) (into the buffer
+        // A's P(j) leaves), B's tile j, S_A(j+2) (into the buffer B's P(j)
+        // leaves): each query tile's next S is ready before its softmax step
+        // ends.
+        // S(w, t) once K_t is here, then its commit.
+        auto next_s = [&](int w, int t) {
+          if (!ok || t >= n_w[w]) return;
+          ok = mbar_wait(b_kfull(t % NK), (t / NK) & 1, abort_flag);
+          if (!ok) return;
+          tc_fence_after();
+          issue_s(w, t, s_col(w, t));
+          umma_commit(b_sfull(w, t));
+        };
+        bool any_kept = false, v_ready = false;
+        // Warpgroup w's tile j: its decision; for a kept tile P_lo V as soon
+        // as P_lo is stored and P_hi V once P is complete, then o_done.
+        auto process = [&](int w, int j, int vs) {
+          if (!ok || j >= n_w[w]) return;
+          if (!(ok = mbar_wait(b_vmma(w, j), pair_par(j), abort_flag))) return;
+          if (!kflag[w * 2 + (j & 1)]) return;
+          any_kept = true;
+          const int k = kc_w[w];
+          if (!(ok = mbar_wait(b_plo(w, k), pair_par(k), abort_flag))) return;
+          if (!v_ready) {
+            if (!(ok = mbar_wait(b_vfull(vs), (kc / NV) & 1, abort_flag))) return;
+            v_ready = true;
+          }
+          tc_fence_after();
+          issue_pv_half(w, s_col(w, j), vs, 0);
+          if (!(ok = mbar_wait(b_phi(w, k), pair_par(k), abort_flag))) return;
+          tc_fence_after();
+          issue_pv_half(w, s_col(w, j), vs, 1);
+          umma_commit(b_odone(w));
+          ++kc_w[w];
+        };
+        next_s(0, 0);
+        next_s(1, 0);
+        next_s(0, 1);
+        if (ok && n_j > 0) umma_commit(b_kempty(0));
+        for (int j = 0; ok && j < n_j; ++j) {
+          const int vs = kc % NV;
+          any_kept = false;
+          v_ready = false;
+          process(0, j, vs);
+          next_s(1, j + 1);
+          process(1, j, vs);
+          next_s(0, j + 2);
+          if (!ok) break;
+          if (any_kept) {
+            umma_commit(b_vempty(vs));
+            ++kc;
+          }
+          if (j + 1 < n_j) umma_commit(b_kempty((j + 1) % NK));
+        }
       }
       // Every MMA issued by this thread completes before the epilogue reads O
       // and before TMEM is released.
@@ -466,8 +534,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int row = row0 + 128 * wg + r;
     const bool row_in = row < p.L;
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
-    const uint32_t tS = tmem + wg * BC + lane_base;
-    const uint32_t tO = tmem + 2 * BC + wg * D + lane_base;
+    const uint32_t tO = tmem + C::kOCol + wg * D + lane_base;
+    int n_kept = 0;  // kept tiles of this query tile so far (parity of o_done)
     const int n_own = wg == 0 ? n_a : n_b;
     int g_tile[NGRP], g_jmax[NGRP];
 #pragma unroll
@@ -508,7 +576,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (elected) post_vote(j, false);
         continue;
       }
-      mbar_wait(b_sfull(wg), j & 1, abort_flag);
+      const uint32_t tS = tmem + s_col(wg, j) + lane_base;
+      mbar_wait(b_sfull(wg, j), pair_par(j), abort_flag);
       tc_fence_after();
       __syncwarp();
       uint32_t sr[BC];
@@ -592,7 +661,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (elected) {
         post_vote(j, tile_kept);
         kflag[wg * 2 + (j & 1)] = tile_kept ? 1 : 0;
-        mbar_arrive(b_vmma(wg));
+        mbar_arrive(b_vmma(wg, j));
       }
       if (!tile_kept) continue;
 
@@ -620,7 +689,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint64_t nref2 = f2pack(nref, nref);
       __syncwarp();
       if (__any_sync(0xffffffffu, rescale)) {
-        // O(j-1) is complete: S(j) was committed after P.V(j-1).
+        // O must hold every earlier P.V.  With one S buffer per query tile it
+        // does: S(j) was committed after P.V(j-1).  With three, S(j) may be
+        // ready first, so wait for the last kept tile's P.V (a rescale needs
+        // an earlier kept tile, so n_kept >= 1).
+        if (TRIPLE) {
+          mbar_wait(b_odone(wg), (n_kept - 1) & 1, abort_flag);
+          tc_fence_after();
+        }
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float o32[32];
@@ -643,7 +719,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (none) {
 #pragma unroll
           for (int i = 0; i < HP; ++i) pk[i] = 0u;
-          if (SPLIT && h == 1) warp_signal(b_hfree(wg));  // its S was read in the max pass
         } else {
           // The row max is known; re-read this half of S (its columns are
           // still intact: P of half h lands in columns [h HP, h HP + HP)).
@@ -655,7 +730,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           } else {
             tmem_wait_ld_tie32(rr);
           }
-          if (SPLIT && h == 1) warp_signal(b_hfree(wg));  // upper S columns free for S_hi(j+1)
           const float* sh = reinterpret_cast<const float*>(rr);
           if (need_mask) {
 #pragma unroll
@@ -688,8 +762,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if constexpr (HP == 32) tmem_st32(tS + h * HP, pk);
         else tmem_st16(tS + h * HP, pk);
         tmem_st_wait();
-        warp_signal(h == 0 ? b_plo(wg) : b_phi(wg));
+        warp_signal(h == 0 ? b_plo(wg, n_kept) : b_phi(wg, n_kept));
       }
+      ++n_kept;
       if (!none) {
         uint64_t sum2 = sum2v[0], sumr2 = sumr2v[0];
 #pragma unroll
