@@ -78,8 +78,15 @@ constexpr int kPfVoteSlots = 4;
 #define SSKIP_PF_SCALAR 0     // scalar instead of packed f32x2 scale / sum
 #endif
 #ifndef SSKIP_PF_RELOAD
-#define SSKIP_PF_RELOAD 1     // reload S from TMEM in 64-column halves for the exponentials
+#define SSKIP_PF_RELOAD 1     // re-read S from TMEM in halves for the exponentials (d = 128)
 #endif
+#ifndef SSKIP_PF_RELOAD_D64
+#define SSKIP_PF_RELOAD_D64 0  // at d = 64 S stays in registers from the max pass
+#endif
+template <int D>
+__device__ __forceinline__ constexpr bool kReload() {
+  return (D == 64 ? SSKIP_PF_RELOAD_D64 : SSKIP_PF_RELOAD) != 0;
+}
 #ifndef SSKIP_PF_NACC
 #define SSKIP_PF_NACC 4       // independent packed accumulators of the row sum
 #endif
@@ -88,6 +95,9 @@ constexpr int kPfVoteSlots = 4;
 #endif
 #ifndef SSKIP_PF_ROUNDED_L
 #define SSKIP_PF_ROUNDED_L 0  // 1: O is divided by the sum of the bf16 P that P.V used
+#endif
+#ifndef SSKIP_PF_ALT
+#define SSKIP_PF_ALT 1        // d = 64 with three S buffers: the two query tiles take turns at their exponentials
 #endif
 #ifndef SSKIP_PF_MMA_NAP
 #define SSKIP_PF_MMA_NAP 0    // ns the MMA thread sleeps after a poll that found nothing to issue
@@ -131,7 +141,7 @@ struct PrefillCfg {
   // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], then per
   // warpgroup s_full[2], vote_mma[2], p_lo[2], p_hi[2], o_done, then
   // vote_full[2][VS], vote_empty[2][VS], mma_done
-  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 9 * 2 + 4 * kPfVoteSlots + 1;
+  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 9 * 2 + 4 * kPfVoteSlots + 1 + 2;
   static constexpr int kMisc = kBar + kNumBars * 8;
   // kept flags [2 wg][2 parity], vote_kept[VS][2], warp vote flags
   // [2 wg][2 parity][4], tmem, abort, warp gaps [2 wg][2 parity][4] (fp32)
@@ -220,17 +230,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     return smem_u32(&bars[kWgBar + 18 + 2 * VS + w * VS + s]);
   };
   const uint32_t b_mmadone = smem_u32(&bars[kWgBar + 18 + 4 * VS]);
+  // Turn token of a query tile's exponentials (one arrival per softmax warp).
+  auto b_tok = [&](int w) { return smem_u32(&bars[kWgBar + 19 + 4 * VS + w]); };
+  constexpr bool ALT = TRIPLE && D == 64 && SSKIP_PF_ALT != 0;
   // TMEM column of the S/P buffer of query tile w at key tile j.
   auto s_col = [&](int w, int j) { return uint32_t((TRIPLE ? (2 * j + w) % 3 : w) * BC); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work unit: 256 rows of one (batch, query head); heaviest causal first.
-  const int bh_count = p.B * p.Hq;
-  const int ublk = blockIdx.x / bh_count;
+  // ---- work unit: 256 rows of one (batch, query head).  CTAs are ordered by
+  // (batch, kv head), then unit (heaviest causal unit first), then the kv
+  // head's G query heads: the CTAs resident at any time mostly read one kv
+  // head's K and V, which then stay in L2 instead of being re-read from HBM
+  // by every unit of every head.
+  const int per_grp = p.n_units * p.G;
+  const int grp = blockIdx.x / per_grp;
+  const int rem = blockIdx.x - grp * per_grp;
+  const int ublk = rem / p.G;
   const int iu = CAUSAL ? (p.n_units - 1 - ublk) : ublk;
-  const int bh = blockIdx.x % bh_count;
-  const int b = bh / p.Hq, hq = bh % p.Hq, kvh = hq / p.G;
+  const int b = grp / p.Hkv, kvh = grp % p.Hkv;
+  const int hq = kvh * p.G + (rem - ublk * p.G);
   const int row0 = iu * kPfUnitRows;
 
   // Key tiles each MMA tile visits (the union over its vote groups).
@@ -261,6 +280,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         mbar_init(b_phi(w, i), 4);
       }
       mbar_init(b_odone(w), 1);
+      mbar_init(b_tok(w), 4);
     }
     for (int w = 0; w < 2; ++w)
       for (int s = 0; s < VS; ++s) { mbar_init(b_vote_full(w, s), 1); mbar_init(b_vote_empty(w, s), 1); }
@@ -571,9 +591,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (lane == 0) mbar_arrive(bar);
     };
 
+    // Turns (ALT): the exponentials of A's tile j follow B's of tile j - 1,
+    // B's of tile j follow A's of tile j; a tile without exponentials passes
+    // its turn at once.  Each warp waits for the other query tile's four
+    // warps and hands its own turn on.
+    auto take_turn = [&](int j) {
+      if (ALT && (wg == 1 || j > 0))
+        mbar_wait(b_tok(1 - wg), (wg == 1 ? j : j - 1) & 1, abort_flag);
+    };
+    auto pass_turn = [&]() {
+      if (ALT) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b_tok(wg));
+      }
+    };
     for (int j = 0; j < n_j; ++j) {
       if (j >= n_own) {  // this tile has no row here: vote "not kept" only
         if (elected) post_vote(j, false);
+        take_turn(j);
+        pass_turn();
         continue;
       }
       const uint32_t tS = tmem + s_col(wg, j) + lane_base;
@@ -663,7 +699,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         kflag[wg * 2 + (j & 1)] = tile_kept ? 1 : 0;
         mbar_arrive(b_vmma(wg, j));
       }
-      if (!tile_kept) continue;
+      if (!tile_kept) {
+        take_turn(j);
+        pass_turn();
+        continue;
+      }
 
       // Block vote: every row of a kept group updates.  Warp vote: only the
       // rows of a warp slice that did not pass.
@@ -713,24 +753,58 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       uint64_t sum2v[SSKIP_PF_NACC], sumr2v[SSKIP_PF_NACC];
 #pragma unroll
       for (int a = 0; a < SSKIP_PF_NACC; ++a) sum2v[a] = sumr2v[a] = f2pack(0.f, 0.f);
+      // P of one half of the keys (HK keys -> HP packed bf16 columns).
+      uint32_t pk[HP];
+      auto exp_half = [&](int h, const float* sh) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {  // HK keys -> HP packed columns at a time
-        uint32_t pk[HP];
-        if (none) {
-#pragma unroll
-          for (int i = 0; i < HP; ++i) pk[i] = 0u;
-        } else {
-          // The row max is known; re-read this half of S (its columns are
-          // still intact: P of half h lands in columns [h HP, h HP + HP)).
-          uint32_t rr[HK];
-          tmem_ld32_async(tS + h * HK, rr);
-          if constexpr (HK == 64) {
-            tmem_ld32_async(tS + h * HK + 32, rr + 32);
-            tmem_wait_ld_tie64(rr);
+        for (int i = 0; i < HP; ++i) {
+          const int c = h * HP + i;  // pair index within the tile
+          float p0, p1;
+          const uint64_t x2 = ffma2(f2pack(sh[2 * i], sh[2 * i + 1]), scale2, nref2);
+          if (exp2_on_fma<D>(c)) {
+            f2unpack(exp2_fma2(x2), p0, p1);
           } else {
-            tmem_wait_ld_tie32(rr);
+            float x0, x1;
+            f2unpack(x2, x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
           }
-          const float* sh = reinterpret_cast<const float*>(rr);
+          sum2v[c % SSKIP_PF_NACC] = fadd2(sum2v[c % SSKIP_PF_NACC], f2pack(p0, p1));
+          pk[i] = pack_bf16x2(p0, p1);
+          if (SSKIP_PF_ROUNDED_L)  // the two bf16 halves widened exactly
+            sumr2v[c % SSKIP_PF_NACC] =
+                fadd2(sumr2v[c % SSKIP_PF_NACC], f2pack(__uint_as_float(pk[i] << 16),
+                                                        __uint_as_float(pk[i] & 0xFFFF0000u)));
+        }
+      };
+      // P of half h lands in columns [h HP, h HP + HP) of the S buffer.
+      auto store_half = [&](int h) {
+        if constexpr (HP == 32) tmem_st32(tS + h * HP, pk);
+        else tmem_st16(tS + h * HP, pk);
+      };
+      if (none) {
+        take_turn(j);
+        pass_turn();
+#pragma unroll
+        for (int i = 0; i < HP; ++i) pk[i] = 0u;
+        store_half(0);
+        tmem_st_wait();
+        warp_signal(b_plo(wg, n_kept));
+        store_half(1);
+        tmem_st_wait();
+        warp_signal(b_phi(wg, n_kept));
+      } else if constexpr (kReload<D>()) {
+        // The row max is known; re-read each half of S (its columns are still
+        // intact: P of the first half lands in the first quarter).  The second
+        // half's load is in flight while P_lo lands.
+        uint32_t rr[HK];
+        auto load_half = [&](int h) {
+          tmem_ld32_async(tS + h * HK, rr);
+          if constexpr (HK == 64) tmem_ld32_async(tS + h * HK + 32, rr + 32);
+        };
+        auto wait_half = [&](int h) {
+          if constexpr (HK == 64) tmem_wait_ld_tie64(rr);
+          else tmem_wait_ld_tie32(rr);
           if (need_mask) {
 #pragma unroll
             for (int c = 0; c < HK; ++c) {
@@ -738,31 +812,33 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               if (key >= p.L || (CAUSAL && key > row)) rr[c] = __float_as_uint(-INFINITY);
             }
           }
-#pragma unroll
-          for (int i = 0; i < HP; ++i) {
-            const int c = h * HP + i;  // pair index within the tile
-            float p0, p1;
-            const uint64_t x2 = ffma2(f2pack(sh[2 * i], sh[2 * i + 1]), scale2, nref2);
-            if (exp2_on_fma<D>(c)) {
-              f2unpack(exp2_fma2(x2), p0, p1);
-            } else {
-              float x0, x1;
-              f2unpack(x2, x0, x1);
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
-            sum2v[c % SSKIP_PF_NACC] = fadd2(sum2v[c % SSKIP_PF_NACC], f2pack(p0, p1));
-            pk[i] = pack_bf16x2(p0, p1);
-            if (SSKIP_PF_ROUNDED_L)  // the two bf16 halves widened exactly
-              sumr2v[c % SSKIP_PF_NACC] =
-                  fadd2(sumr2v[c % SSKIP_PF_NACC], f2pack(__uint_as_float(pk[i] << 16),
-                                                          __uint_as_float(pk[i] & 0xFFFF0000u)));
-          }
-        }
-        if constexpr (HP == 32) tmem_st32(tS + h * HP, pk);
-        else tmem_st16(tS + h * HP, pk);
+        };
+        load_half(0);
+        take_turn(j);
+        wait_half(0);
+        exp_half(0, reinterpret_cast<const float*>(rr));
+        store_half(0);
+        load_half(1);
         tmem_st_wait();
-        warp_signal(h == 0 ? b_plo(wg, n_kept) : b_phi(wg, n_kept));
+        warp_signal(b_plo(wg, n_kept));
+        wait_half(1);
+        exp_half(1, reinterpret_cast<const float*>(rr));
+        pass_turn();
+        store_half(1);
+        tmem_st_wait();
+        warp_signal(b_phi(wg, n_kept));
+      } else {
+        // S stays in registers from the max pass (already masked).
+        take_turn(j);
+        exp_half(0, s);
+        store_half(0);
+        tmem_st_wait();
+        warp_signal(b_plo(wg, n_kept));
+        exp_half(1, s + HK);
+        pass_turn();
+        store_half(1);
+        tmem_st_wait();
+        warp_signal(b_phi(wg, n_kept));
       }
       ++n_kept;
       if (!none) {
