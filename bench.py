@@ -573,8 +573,8 @@ def report(args, w, dw, world, legs, ms, ms_dense, ems, io_bytes, peaks, peak_ki
             "frac": achieved / peak, "traffic": ncu_traffic("prefill_kernel"),
             "kernel": f"prefill_kernel<{w.d},{w.Br},{w.Bc},{'causal' if w.causal else 'full'}>",
             "leg": head["key"],
-            "peak_source": f"{peak_kind} bf16_tflops (burst; the SM clock stays at its maximum "
-                           f"during the step)"}
+            "peak_source": f"{peak_kind} bf16_tflops (burst, the conservative figure; the SM "
+                           f"clock seen during the step is under clocks)"}
         line["prefill"] = pre
         if head["name"] in ems:
             line["e2e"] = {"value": world * hs["executed"] / (ems[head["name"]] / 1e3) / 1e12,
