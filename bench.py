@@ -831,16 +831,27 @@ def run_reorder(args):
     for order, (qq, kk, vv, oo, ll) in (("raster", (q, k, v, o, lse)),
                                         ("hilbert", (qp, kp, vp, op, lsep))):
         for vote in (w.Br, 32):
-            def run(f=w.tsf):
-                sk.sskip_attn_prefill_vote(qq, kk, vv, oo, ll, causal=w.causal,
-                                           sm_scale=w.scale, threshold_scale_factor=f, Br=w.Br,
-                                           Bc=w.Bc, vote_rows=vote, counts=cnt)
+            # The block vote runs the plain kernel; the per-warp vote its own
+            # instantiation (sskip_attn_prefill_vote), timed against a dense
+            # control of that same instantiation.
+            def run(f=w.tsf, vote=vote):
+                if vote == w.Br:
+                    sk.sskip_attn_prefill(qq, kk, vv, oo, ll, causal=w.causal, sm_scale=w.scale,
+                                          threshold_scale_factor=f, Br=w.Br, Bc=w.Bc,
+                                          skip_count=cnt)
+                else:
+                    sk.sskip_attn_prefill_vote(qq, kk, vv, oo, ll, causal=w.causal,
+                                               sm_scale=w.scale, threshold_scale_factor=f,
+                                               Br=w.Br, Bc=w.Bc, vote_rows=vote, counts=cnt)
             run()
             c = cnt.cpu().tolist()
             ms = time_it(run)
+            ms0 = time_it(lambda: run(0.0))
             f = prefill_flops(w, c[1], c[0])
-            rows.append({"order": order, "vote_rows": vote, "ms": ms,
-                         "skip_fraction": c[0] / c[1], "slice_skip_fraction": c[2] / c[3],
+            rows.append({"order": order, "vote_rows": vote, "ms": ms, "ms_dense": ms0,
+                         "speedup_vs_dense": ms0 / ms,
+                         "skip_fraction": c[0] / c[1],
+                         "slice_skip_fraction": (c[2] / c[3]) if vote != w.Br else c[0] / c[1],
                          "executed_tflops": f["executed"] / ms / 1e9,
                          "executed_frac_of_peak": f["executed"] / ms / 1e9 / peak,
                          "dense_equiv_tflops": f["dense"] / ms / 1e9})

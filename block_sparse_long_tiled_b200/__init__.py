@@ -25,7 +25,9 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libsskip_attn.so")
 
-SSKIP_OK, SSKIP_ERR_INVALID_ARG, SSKIP_ERR_UNSUPPORTED, SSKIP_ERR_CUDA, SSKIP_ERR_TIMEOUT = range(5)
+(SSKIP_OK, SSKIP_ERR_INVALID_ARG, SSKIP_ERR_UNSUPPORTED, SSKIP_ERR_CUDA, SSKIP_ERR_TIMEOUT,
+ SSKIP_ERR_DEVICE_CHECK) = range(6)
+LIB_DEBUG_PATH = os.path.join(_PKG, "libsskip_attn_debug.so")
 
 EXPORTS = ("sskip_version", "sskip_status_string", "sskip_device_supported",
            "sskip_attn_prefill", "sskip_attn_prefill_ex", "sskip_attn_prefill_vote",
@@ -47,62 +49,77 @@ class SSkipError(RuntimeError):
 
 
 _lib = None
+_lib_debug = None
 
 
 def lib() -> ctypes.CDLL:
     """Load libsskip_attn.so (build it first with block_sparse_long_tiled_b200.build)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
-                               "`python -m block_sparse_long_tiled_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
-        P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
-        L.sskip_version.restype = I
-        L.sskip_version.argtypes = []
-        L.sskip_status_string.restype = ctypes.c_char_p
-        L.sskip_status_string.argtypes = [I]
-        L.sskip_device_supported.restype = I
-        L.sskip_device_supported.argtypes = [I]
-        pre = [P, P, P, P, P, I, I, I, I, I, I, F, F, I, I, P]
-        L.sskip_attn_prefill.restype = I
-        L.sskip_attn_prefill.argtypes = pre + [P]
-        L.sskip_attn_prefill_ex.restype = I
-        L.sskip_attn_prefill_ex.argtypes = pre[:-1] + [P, P, P]
-        L.sskip_attn_prefill_vote.restype = I
-        L.sskip_attn_prefill_vote.argtypes = pre[:-1] + [I, P, P, P, P, P]
-        L.sskip_attn_decode_workspace_size.restype = Z
-        L.sskip_attn_decode_workspace_size.argtypes = [I, I, I, I]
-        dec = [P, P, P, P, P, P, I, I, I, I, I, F, F, I, I, P, Z, P]
-        L.sskip_attn_decode.restype = I
-        L.sskip_attn_decode.argtypes = dec + [P]
-        L.sskip_attn_decode_ex.restype = I
-        L.sskip_attn_decode_ex.argtypes = dec + [P, P]
-        L.sskip_attn_decode_crit.restype = I
-        L.sskip_attn_decode_crit.argtypes = dec + [P, P, P]
-        D = ctypes.c_double
-        L.sskip_calibrate_factor.restype = I
-        L.sskip_calibrate_factor.argtypes = [P, Z, D, D, P, P, P]
-        L.sskip_hilbert3d_order.restype = I
-        L.sskip_hilbert3d_order.argtypes = [I, I, I, I, P]
-        L.sskip_permute_rows.restype = I
-        L.sskip_permute_rows.argtypes = [P, P, P, ctypes.c_longlong, I, I, I, P]
-        L.sskip_attn_prefill_host.restype = I
-        L.sskip_attn_prefill_host.argtypes = [P] * 10 + [I, I, I, I, I, I, F, F, I, I, I, P, P]
-        L.sskip_attn_decode_host.restype = I
-        L.sskip_attn_decode_host.argtypes = [P] * 10 + [I, I, I, I, I, F, F, I, I, P, Z, P, P]
-        L.sskip_attn_step.restype = I
-        L.sskip_attn_step.argtypes = ([P, P, P, P, P, I, I, I, I, I, P] +
-                                      [P, P, P, P, P, P, I, I, I, P, Z, P] +
-                                      [I, I, I, F, F, F, P])
-        L.sskip_attn_decode_noalloc.restype = I
-        L.sskip_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, F, I, I, P, P]
-        L.sskip_get_status.restype = I
-        L.sskip_get_status.argtypes = [P]
-        L.sskip_selftest_watchdog.restype = I
-        L.sskip_selftest_watchdog.argtypes = [ctypes.c_uint, P]
-        _lib = L
+        _lib = _load(LIB_PATH)
     return _lib
+
+
+def debug_lib() -> ctypes.CDLL:
+    """Load libsskip_attn_debug.so: the same C ABI with device-side index
+    checks (a failed one latches SSKIP_ERR_DEVICE_CHECK). Its status word is
+    its own: read it with debug_lib().sskip_get_status."""
+    global _lib_debug
+    if _lib_debug is None:
+        _lib_debug = _load(LIB_DEBUG_PATH)
+    return _lib_debug
+
+
+def _load(path: str) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m block_sparse_long_tiled_b200.build`")
+    L = ctypes.CDLL(path)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.sskip_version.restype = I
+    L.sskip_version.argtypes = []
+    L.sskip_status_string.restype = ctypes.c_char_p
+    L.sskip_status_string.argtypes = [I]
+    L.sskip_device_supported.restype = I
+    L.sskip_device_supported.argtypes = [I]
+    pre = [P, P, P, P, P, I, I, I, I, I, I, F, F, I, I, P]
+    L.sskip_attn_prefill.restype = I
+    L.sskip_attn_prefill.argtypes = pre + [P]
+    L.sskip_attn_prefill_ex.restype = I
+    L.sskip_attn_prefill_ex.argtypes = pre[:-1] + [P, P, P]
+    L.sskip_attn_prefill_vote.restype = I
+    L.sskip_attn_prefill_vote.argtypes = pre[:-1] + [I, P, P, P, P, P]
+    L.sskip_attn_decode_workspace_size.restype = Z
+    L.sskip_attn_decode_workspace_size.argtypes = [I, I, I, I]
+    dec = [P, P, P, P, P, P, I, I, I, I, I, F, F, I, I, P, Z, P]
+    L.sskip_attn_decode.restype = I
+    L.sskip_attn_decode.argtypes = dec + [P]
+    L.sskip_attn_decode_ex.restype = I
+    L.sskip_attn_decode_ex.argtypes = dec + [P, P]
+    L.sskip_attn_decode_crit.restype = I
+    L.sskip_attn_decode_crit.argtypes = dec + [P, P, P]
+    D = ctypes.c_double
+    L.sskip_calibrate_factor.restype = I
+    L.sskip_calibrate_factor.argtypes = [P, Z, D, D, P, P, P]
+    L.sskip_hilbert3d_order.restype = I
+    L.sskip_hilbert3d_order.argtypes = [I, I, I, I, P]
+    L.sskip_permute_rows.restype = I
+    L.sskip_permute_rows.argtypes = [P, P, P, ctypes.c_longlong, I, I, I, P]
+    L.sskip_attn_prefill_host.restype = I
+    L.sskip_attn_prefill_host.argtypes = [P] * 10 + [I, I, I, I, I, I, F, F, I, I, I, P, P]
+    L.sskip_attn_decode_host.restype = I
+    L.sskip_attn_decode_host.argtypes = [P] * 10 + [I, I, I, I, I, F, F, I, I, P, Z, P, P]
+    L.sskip_attn_step.restype = I
+    L.sskip_attn_step.argtypes = ([P, P, P, P, P, I, I, I, I, I, P] +
+                                  [P, P, P, P, P, P, I, I, I, P, Z, P] +
+                                  [I, I, I, F, F, F, P])
+    L.sskip_attn_decode_noalloc.restype = I
+    L.sskip_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, F, I, I, P, P]
+    L.sskip_get_status.restype = I
+    L.sskip_get_status.argtypes = [P]
+    L.sskip_selftest_watchdog.restype = I
+    L.sskip_selftest_watchdog.argtypes = [ctypes.c_uint, P]
+    return L
 
 
 def status_string(status: int) -> str:

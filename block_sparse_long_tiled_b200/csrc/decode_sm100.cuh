@@ -143,6 +143,9 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
   const int j0 = split * c_per;
   const int ntiles = max(0, min(n_k, j0 + c_per) - j0);
   const size_t head0 = (size_t)b * p.Hq + (size_t)kvh * G;
+  if (!dev_check(b < p.B && kvh < p.Hkv && split < p.S && head0 + G <= (size_t)p.B * p.Hq &&
+                 kvh * G + G <= p.Hq))
+    return;  // the whole CTA, before any barrier
 
   if (ntiles == 0) {  // an empty split contributes nothing to the merge
     for (int i = tid; i < G * D; i += kDecThreads)
@@ -177,6 +180,10 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
 
   auto issue = [&](uint32_t ring, int stage, uint32_t bar, const __nv_bfloat16* base, int t) {
     const uint32_t bytes = (uint32_t)tile_keys(t) * D * 2;
+    if (!dev_check(j0 + t < n_k && (j0 + t) * kDecBc + tile_keys(t) <= p.Lmax && bytes > 0)) {
+      mbar_arrive(bar);  // the phase completes without data
+      return;
+    }
     mbar_arrive_expect_tx(bar, bytes);
     bulk_load(ring + stage * L::kTileBytes, base + (size_t)(j0 + t) * kDecBc * D, bytes, bar);
   };
@@ -297,7 +304,7 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
                     : (m_run == -INFINITY) ? INFINITY : m_loc - m_run;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) gap = fmaxf(gap, __shfl_xor_sync(0xffffffffu, gap, o));
-        if (lane == 0)
+        if (lane == 0 && dev_check(j0 + t < p.n_k_max))
           p.tile_crit[((size_t)b * p.Hkv + kvh) * p.n_k_max + j0 + t] =
               gap * 0.69314718055994531f + logf((float)Lb);
       }
@@ -321,7 +328,7 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
         kept_mask &= ~(1ull << (t & 63));
         n_skipped += 1;
       }
-      if (tid == 0 && p.tile_state)
+      if (tid == 0 && p.tile_state && dev_check(j0 + t < p.n_k_max))
         p.tile_state[((size_t)b * p.Hkv + kvh) * p.n_k_max + j0 + t] = skip ? 2 : 1;
     }
 
@@ -437,6 +444,7 @@ __global__ void __launch_bounds__(kDecThreads, dec_ctas_per_sm<D, G>())
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
   const size_t bh = blockIdx.x;
+  if (!dev_check(bh < (size_t)p.B * p.Hq)) return;
   const float* lp = p.lse_part + bh * p.S;
   __shared__ float w_s[64];
   __shared__ float lse_s;

@@ -99,6 +99,12 @@ __device__ __forceinline__ constexpr bool kReload() {
 #ifndef SSKIP_PF_ALT
 #define SSKIP_PF_ALT 1        // d = 64 with three S buffers: the two query tiles take turns at their exponentials
 #endif
+#ifndef SSKIP_PF_EXT_RELOAD
+#define SSKIP_PF_EXT_RELOAD 1  // the per-warp-vote build re-reads S at every d
+#endif
+#ifndef SSKIP_PF_ALT_D128
+#define SSKIP_PF_ALT_D128 0   // the same turn-taking with one S buffer per query tile
+#endif
 #ifndef SSKIP_PF_MMA_NAP
 #define SSKIP_PF_MMA_NAP 0    // ns the MMA thread sleeps after a poll that found nothing to issue
 #endif
@@ -232,7 +238,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t b_mmadone = smem_u32(&bars[kWgBar + 18 + 4 * VS]);
   // Turn token of a query tile's exponentials (one arrival per softmax warp).
   auto b_tok = [&](int w) { return smem_u32(&bars[kWgBar + 19 + 4 * VS + w]); };
-  constexpr bool ALT = TRIPLE && D == 64 && SSKIP_PF_ALT != 0;
+  constexpr bool ALT = (TRIPLE && D == 64 && SSKIP_PF_ALT != 0) || (!TRIPLE && SSKIP_PF_ALT_D128 != 0);
   // TMEM column of the S/P buffer of query tile w at key tile j.
   auto s_col = [&](int w, int j) { return uint32_t((TRIPLE ? (2 * j + w) % 3 : w) * BC); };
 
@@ -267,6 +273,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   };
   const int n_a = tiles_visited(0), n_b = tiles_visited(1);
   const int n_j = max(n_a, n_b);
+  // (Every thread computes the same unit, so all return together, before
+  // any barrier.)
+  if (!dev_check(b < p.B && hq < p.Hq && kvh < p.Hkv && iu < p.n_units && row0 < p.L &&
+                 n_j <= p.n_k))
+    return;
+  static_assert(C::kOCol + 2 * D <= C::kTmemCols, "TMEM columns");
 
   if (threadIdx.x == 0) {
     mbar_init(b_qfull, 1);
@@ -314,6 +326,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       for (int j = 0; j < n_j; ++j) {
         const int s = j % NK;
         if (j >= NK && !mbar_wait(b_kempty(s), ((j / NK) - 1) & 1, abort_flag)) break;
+        if (!dev_check(j < p.n_k && b * p.Hkv + kvh < p.B * p.Hkv)) {
+          mbar_arrive(b_kfull(s));  // the phase completes without data
+          continue;
+        }
         mbar_arrive_expect_tx(b_kfull(s), C::kKVBytes);
 #pragma unroll
         for (int blk = 0; blk < D / 64; ++blk)
@@ -522,11 +538,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (kept_any && !issued) {
             const int vs = kc % NV;
             if (kc >= NV && !mbar_wait(b_vempty(vs), ((kc / NV) - 1) & 1, abort_flag)) break;
-            mbar_arrive_expect_tx(b_vfull(vs), C::kKVBytes);
+            if (!dev_check(j < p.n_k && vs < NV)) {
+              mbar_arrive(b_vfull(vs));  // the phase completes without data
+            } else {
+              mbar_arrive_expect_tx(b_vfull(vs), C::kKVBytes);
 #pragma unroll
-            for (int blk = 0; blk < D / 64; ++blk)
-              tma_load_3d(sbase + C::kV + vs * C::kKVBytes + blk * BC * 128, &tmV, b_vfull(vs),
-                          blk * 64, j * BC, b * p.Hkv + kvh);
+              for (int blk = 0; blk < D / 64; ++blk)
+                tma_load_3d(sbase + C::kV + vs * C::kKVBytes + blk * BC * 128, &tmV, b_vfull(vs),
+                            blk * 64, j * BC, b * p.Hkv + kvh);
+            }
             issued = true;
             last = kc++;
           }
@@ -674,9 +694,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         g_kept[g] = vis && !all;
         tile_kept = tile_kept || g_kept[g];
         if (elected && vis) {
+          const size_t rec = (((size_t)b * p.Hq + hq) * p.n_q + g_tile[g]) * p.n_k + j;
+          if (!dev_check(g_tile[g] < p.n_q && j < p.n_k &&
+                         rec < (size_t)p.B * p.Hq * p.n_q * p.n_k))
+            continue;
           ++n_vis;
           n_skip += all ? 1 : 0;
-          const size_t rec = (((size_t)b * p.Hq + hq) * p.n_q + g_tile[g]) * p.n_k + j;
           if (p.tile_state) p.tile_state[rec] = all ? 2 : 1;
           if (EXT && p.slice_mask)
             p.slice_mask[rec] = uint8_t(0x80u | (p.slice_vote ? bits : (all ? 1u : 0u)));
@@ -793,7 +816,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         store_half(1);
         tmem_st_wait();
         warp_signal(b_phi(wg, n_kept));
-      } else if constexpr (kReload<D>()) {
+      } else if constexpr (kReload<D>() || (EXT && SSKIP_PF_EXT_RELOAD)) {
         // The row max is known; re-read each half of S (its columns are still
         // intact: P of the first half lands in the first quarter).  The second
         // half's load is in flight while P_lo lands.
@@ -860,7 +883,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     mbar_wait(b_mmadone, 0, abort_flag);
     tc_fence_after();
     __syncwarp();
-    const bool store = row_in && my_jmax >= 0 && n_own > 0 && l_run > 0.f;
+    const bool store = row_in && my_jmax >= 0 && n_own > 0 && l_run > 0.f &&
+                       dev_check(row < p.L && hq < p.Hq);
     if (n_own > 0) {
       const float inv_l = store ? 1.f / (SSKIP_PF_ROUNDED_L ? lr_run : l_run) : 0.f;
       __nv_bfloat16* orow = p.o + (((size_t)b * p.Hq + hq) * p.L + (store ? row : 0)) * D;

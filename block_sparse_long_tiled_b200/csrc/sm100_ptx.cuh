@@ -19,11 +19,28 @@ __device__ int g_status;
 
 constexpr int kStatusInvalidArg = 1;  // SSKIP_ERR_INVALID_ARG: a device-side argument check failed
 constexpr int kStatusTimeout = 4;     // SSKIP_ERR_TIMEOUT: a bounded wait ran out
+constexpr int kStatusDeviceCheck = 5; // SSKIP_ERR_DEVICE_CHECK: a debug-build index check failed
 // A single wait on an mbarrier never legitimately takes more than microseconds
 // here; one second is far beyond that yet keeps a stuck kernel short.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 __device__ __forceinline__ void latch_status(int code) { atomicCAS(&g_status, 0, code); }
+
+// Debug builds (SSKIP_DEBUG_CHECKS=1, libsskip_attn_debug.so) check tile,
+// ring and record indices on the device.  A failed check latches
+// SSKIP_ERR_DEVICE_CHECK and the caller skips the access (a producer still
+// completes its barrier phase, so no wait is left hanging); nothing traps.
+// In the release build every check is `true` and compiles away.
+#ifndef SSKIP_DEBUG_CHECKS
+#define SSKIP_DEBUG_CHECKS 0
+#endif
+__device__ __forceinline__ bool dev_check(bool ok) {
+  if (SSKIP_DEBUG_CHECKS && !ok) {
+    latch_status(kStatusDeviceCheck);
+    return false;
+  }
+  return true;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

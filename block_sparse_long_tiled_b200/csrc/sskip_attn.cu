@@ -140,6 +140,7 @@ SSKIP_API const char* sskip_status_string(int status) {
     case SSKIP_ERR_UNSUPPORTED: return "unsupported configuration";
     case SSKIP_ERR_CUDA: return "CUDA error";
     case SSKIP_ERR_TIMEOUT: return "device-side wait timed out";
+    case SSKIP_ERR_DEVICE_CHECK: return "device-side index check failed (debug build)";
     default: return "unknown status";
   }
 }

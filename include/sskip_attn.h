@@ -39,6 +39,12 @@
  *    or index) are latched in a per-device status
  *    word that sskip_get_status() reads.  No C++ exception crosses this ABI.
  *  - Outputs, the counters included, are overwritten, never accumulated.
+ *  - Debug build.  libsskip_attn_debug.so exports the same functions from the
+ *    same sources compiled with device-side checks of tile, ring and record
+ *    indices (a stand-in for a memory checker).  A failed check latches
+ *    SSKIP_ERR_DEVICE_CHECK in the status word and skips the access; a
+ *    producer still completes its barrier phase, so nothing traps or hangs.
+ *    Outputs are bit-identical to the release build's when no check fails.
  */
 #ifndef SSKIP_ATTN_H_
 #define SSKIP_ATTN_H_
@@ -55,7 +61,9 @@ typedef enum {
     SSKIP_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, misaligned, tsf < 0 */
     SSKIP_ERR_UNSUPPORTED = 2,  /* valid but not built: d, tile sizes, device  */
     SSKIP_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed        */
-    SSKIP_ERR_TIMEOUT = 4       /* a bounded device-side wait ran out          */
+    SSKIP_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out          */
+    SSKIP_ERR_DEVICE_CHECK = 5  /* a device-side index check of the debug
+                                   build failed (libsskip_attn_debug.so)       */
 } sskip_status;
 
 /* Library version (major * 10000 + minor * 100 + patch). */

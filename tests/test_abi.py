@@ -38,9 +38,18 @@ def test_library_exports_every_declared_symbol(lib):
     assert lib.sskip_version() == 100
 
 
+def test_debug_library_exports_the_same_api(lib):
+    dbg = sk.debug_lib()
+    for name in header_functions():
+        assert hasattr(dbg, name), name
+    assert dbg.sskip_version() == lib.sskip_version()
+    assert dbg.sskip_status_string(sk.SSKIP_ERR_DEVICE_CHECK).decode().startswith("device-side index")
+
+
 def test_status_strings(lib):
     assert sk.status_string(0) == "ok"
     assert "timed out" in sk.status_string(4)
+    assert "debug build" in sk.status_string(5)
     assert sk.status_string(99) == "unknown status"
 
 
