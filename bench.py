@@ -524,6 +524,8 @@ def leg_oracle_baseline(leg) -> dict:
 def report(args, w, dw, world, legs, ms, ms_dense, ems, io_bytes, peaks, peak_kind,
            clock_rec) -> dict:
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sustained = float(peaks.get("bf16_tflops_sustained",
+                                     FALLBACK_PEAKS["bf16_tflops_sustained"]))
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     K = args.steps
     line = {"metric": METRIC, "value": None, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
@@ -571,6 +573,7 @@ def report(args, w, dw, world, legs, ms, ms_dense, ems, io_bytes, peaks, peak_ki
         line["roofline"] = {
             "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": ncu_traffic("prefill_kernel"),
+            "frac_of_sustained": achieved / peak_sustained,
             "kernel": f"prefill_kernel<{w.d},{w.Br},{w.Bc},{'causal' if w.causal else 'full'}>",
             "leg": head["key"],
             "peak_source": f"{peak_kind} bf16_tflops (burst, the conservative figure; the SM "
@@ -677,6 +680,14 @@ def run_calibration(args):
         torch.bfloat16)
     targets = [float(t) for t in args.targets.split(",") if t]
 
+    def _unreachable_text(e) -> str:
+        # SSKIP_ERR_UNSUPPORTED from the selection: no factor below the
+        # smallest context length skips that share (the record holds only
+        # while t = factor / L < 1).
+        if getattr(e, "status", None) == sk.SSKIP_ERR_UNSUPPORTED:
+            return "no factor below the context length reaches this share (t must stay < 1)"
+        return str(e)
+
     def time_it(fn):
         ts = []
         for i in range(args.warmup + args.steps):
@@ -711,7 +722,7 @@ def run_calibration(args):
                                          target_ratio=tgt, Br=w.Br, Bc=w.Bc)
             except sk.SSkipError as e:
                 print(json.dumps({"calibration": w.name, "reading": rd, "target": tgt,
-                                  "unreachable": str(e)}), flush=True)
+                                  "unreachable": _unreachable_text(e)}), flush=True)
                 continue
             cal_s = time.perf_counter() - t0
             ms = time_it(lambda: run(r["factor"]))
@@ -755,7 +766,7 @@ def run_calibration(args):
                                         Bc=dw.Bc, num_splits=dw.num_splits)
             except sk.SSkipError as e:
                 print(json.dumps({"calibration": dw.name, "reading": rd, "target": tgt,
-                                  "unreachable": str(e)}), flush=True)
+                                  "unreachable": _unreachable_text(e)}), flush=True)
                 continue
             cal_s = time.perf_counter() - t0
             run_d(r["factor"], tiles)
