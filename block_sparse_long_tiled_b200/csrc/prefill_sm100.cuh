@@ -17,16 +17,18 @@
 //               NK-stage ring (K is needed for every visited tile).
 //   warp 1      TMEM allocator; one thread issues every tcgen05.mma:
 //               per key tile j: P_A.V_j, S_A(j+1), P_B.V_j, S_B(j+1).
-//   warp 2      V producer: watches both warpgroups' votes on tile j and
-//               issues the V_j TMA on the first "keep"; a tile both skip
-//               never loads V.
+//   warp 2      collector: reads both warpgroups' votes on tile j, issues
+//               the V_j TMA on the first "keep" (a tile both skip never
+//               loads V) and writes the tile records and counts.
 //   warps 4..7  softmax of tile A, thread r = TMEM lane r = query row r.
 //   warps 8..11 softmax of tile B.
-// A softmax warpgroup, per key tile: loads its S row from TMEM, masks it,
-// takes the row max, votes (skip iff every valid row of a Br-row query tile
-// passes), posts the vote, and for a kept tile computes P = exp2(S - m) in
-// fp32, packs it to bf16 in place of S in TMEM, and releases the tile to the
-// MMA thread, which runs O += P V with P read straight from TMEM.
+// A softmax warp, per key tile: loads its S rows from TMEM, masks them, takes
+// the row maxima and its vote flag (do all its rows pass?), and posts it.
+// The tile is skipped iff every valid row of a Br-row query tile passes; a
+// warp with a row that did not pass knows the tile is kept without waiting
+// for the others.  For a kept tile it computes P = exp2(S - m) in fp32,
+// packs it to bf16 in place of S in TMEM, and releases the tile to the MMA
+// thread, which runs O += P V with P read straight from TMEM.
 // Skipped tiles cost one QK^T MMA and one row max: no exp, no P, no V bytes.
 //
 // Exponent reference: the vote always uses the exact running max m_run; the
@@ -71,12 +73,6 @@ constexpr int kPfVoteSlots = 4;
 #ifndef SSKIP_PF_FMA_EXP
 #define SSKIP_PF_FMA_EXP 0   // element pairs per 8 whose exp2 runs on the FMA pipe
 #endif
-#ifndef SSKIP_PF_PACK_PRMT
-#define SSKIP_PF_PACK_PRMT 0  // bf16 packing by byte permute instead of cvt
-#endif
-#ifndef SSKIP_PF_SCALAR
-#define SSKIP_PF_SCALAR 0     // scalar instead of packed f32x2 scale / sum
-#endif
 #ifndef SSKIP_PF_RELOAD
 #define SSKIP_PF_RELOAD 1     // re-read S from TMEM in halves for the exponentials (d = 128)
 #endif
@@ -90,23 +86,14 @@ __device__ __forceinline__ constexpr bool kReload() {
 #ifndef SSKIP_PF_NACC
 #define SSKIP_PF_NACC 4       // independent packed accumulators of the row sum
 #endif
-#ifndef SSKIP_PF_TRIPLE
-#define SSKIP_PF_TRIPLE 1     // three rotating S buffers where TMEM has room (3 Bc + 2 d <= 512)
-#endif
 #ifndef SSKIP_PF_ROUNDED_L
 #define SSKIP_PF_ROUNDED_L 0  // 1: O is divided by the sum of the bf16 P that P.V used
-#endif
-#ifndef SSKIP_PF_ALT
-#define SSKIP_PF_ALT 1        // d = 64 with three S buffers: the two query tiles take turns at their exponentials
 #endif
 #ifndef SSKIP_PF_EXT_RELOAD
 #define SSKIP_PF_EXT_RELOAD 1  // the per-warp-vote build re-reads S at every d
 #endif
-#ifndef SSKIP_PF_ALT_D128
-#define SSKIP_PF_ALT_D128 0   // the same turn-taking with one S buffer per query tile
-#endif
-#ifndef SSKIP_PF_MMA_NAP
-#define SSKIP_PF_MMA_NAP 0    // ns the MMA thread sleeps after a poll that found nothing to issue
+#ifndef SSKIP_PF_PRODUCER_REGS
+#define SSKIP_PF_PRODUCER_REGS 88  // registers of the producer, MMA and collector warps (<= 88 with 208)
 #endif
 #ifndef SSKIP_PF_FMA_EXP_D64
 #define SSKIP_PF_FMA_EXP_D64 SSKIP_PF_FMA_EXP  // the same, for head dim 64
@@ -118,13 +105,6 @@ template <int D>
 __device__ __forceinline__ constexpr bool exp2_on_fma(int pair) {
   constexpr int n = D == 64 ? SSKIP_PF_FMA_EXP_D64 : SSKIP_PF_FMA_EXP;
   return n > 0 && ((pair & 7) * n) % 8 < n;
-}
-// Byte-permute packing rounds each (non-negative) P to bf16 half-up: add half
-// a bf16 unit in the last place to the fp32 bits, keep the top 16 bits.  It
-// differs from round-to-nearest-even only at exact ties and runs on the
-// integer ALU instead of the conversion unit.
-__device__ __forceinline__ uint32_t pack_bf16x2_halfup(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 constexpr float kPackBias = 0.0f;
 
@@ -139,19 +119,14 @@ struct PrefillCfg {
   static constexpr int kK = kQ + 2 * kQBytes;
   static constexpr int kV = kK + kNK * kKVBytes;
   static constexpr int kBar = kV + kNV * kKVBytes;
-  // Three S/P buffers that rotate over the two query tiles' key tiles when
-  // TMEM holds them next to the two O accumulators; else one per query tile.
-  static constexpr bool kTriple = SSKIP_PF_TRIPLE != 0 && 3 * BC + 2 * D <= 512;
-  static constexpr int kSBufs = kTriple ? 3 : 2;
-  static constexpr int kOCol = kSBufs * BC;  // first TMEM column of O_A (O_B follows)
+  // One S/P buffer of Bc columns per query tile, then O_A and O_B.
+  static constexpr int kOCol = 2 * BC;  // first TMEM column of O_A (O_B follows)
   // q_full, k_full[NK], k_empty[NK], v_full[NV], v_empty[NV], then per
-  // warpgroup s_full[2], vote_mma[2], p_lo[2], p_hi[2], o_done, then
-  // vote_full[2][VS], vote_empty[2][VS], mma_done
-  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 9 * 2 + 4 * kPfVoteSlots + 1 + 2;
+  // warpgroup s_full, p_lo, p_hi, then vote[2][VS], vote_read[2][VS], mma_done
+  static constexpr int kNumBars = 1 + 2 * kNK + 2 * kNV + 3 * 2 + 4 * kPfVoteSlots + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
-  // kept flags [2 wg][2 parity], vote_kept[VS][2], warp vote flags
-  // [2 wg][2 parity][4], tmem, abort, warp gaps [2 wg][2 parity][4] (fp32)
-  static constexpr int kMiscInts = 4 + 2 * kPfVoteSlots + 16 + 2 + 16;
+  // warp vote flags [2 wg][VS][4], warp gaps [2 wg][VS][4] (fp32), tmem, abort
+  static constexpr int kMiscInts = 16 * kPfVoteSlots + 2;
   static constexpr int kTotal = kMisc + kMiscInts * 4;
   static constexpr int kAlloc = kTotal + 1024;  // room to align the base to 1 KB
   static constexpr int kTmemCols = (kOCol + 2 * D) <= 256 ? 256 : 512;
@@ -163,20 +138,15 @@ struct PrefillCfg {
 // EXT = true adds the per-warp vote, the slice and critical-value records and
 // the four counters (kept out of the plain kernel, which they slow down).
 //
-// Both contractions of a tile run as two halves of Bc/2 keys, so that the
-// tensor core never waits for a whole softmax step (S and P share the
-// Bc TMEM columns of a query tile; P of key tile j, bf16, fills the first
-// Bc/2 columns):
-//   S_hi(j+1) = Q K_{j+1}[Bc/2:]^T  as soon as the softmax has re-read the
-//                                    upper S columns of tile j;
-//   O += P_lo(j) V_j[:Bc/2]         as soon as P of the first half is stored;
-//   O += P_hi(j) V_j[Bc/2:], then S_lo(j+1) = Q K_{j+1}[:Bc/2]^T
-//                                    when the whole P(j) is stored.
-// Only the last pair sits between two softmax steps of a query tile.  A
-// skipped tile releases its S columns right after the vote and the next S
-// follows at once.  tcgen05 MMAs of one thread complete in issue order, so
-// S_lo(j+1) (issued after P.V(j)) is the commit that makes S(j+1) and O
-// visible together.
+// A kept tile's P (bf16) is stored over the first Bc/2 of its S columns in
+// two halves of Bc/2 keys, and P.V runs as two matching halves:
+//   O += P_lo(j) V_j[:Bc/2]   as soon as P of the first half is stored;
+//   O += P_hi(j) V_j[Bc/2:]   once all of P is stored.
+// With one S buffer per query tile, S(j+1) = Q K_{j+1}^T then goes to the
+// same columns: tcgen05 MMAs of one thread complete in issue order, so S(j+1)
+// never overwrites a P that P.V still reads, and its commit makes S(j+1) and
+// O visible together.  A skipped tile releases its S columns at the vote and
+// the next S follows at once.
 template <int D, int BR, int BC, bool CAUSAL, bool EXT>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -187,7 +157,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   constexpr int WPG = BR / 32;    // warps per vote group
   constexpr int HK = BC / 2;      // keys per half tile
   constexpr int HP = HK / 2;      // packed bf16 P columns per half tile
-  constexpr bool TRIPLE = C::kTriple;
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BC, 0, 0);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
   static_assert(BR == 64 || BR == 128, "Br");
@@ -198,12 +167,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBar);
   int* misc = reinterpret_cast<int*>(smem + C::kMisc);
-  volatile int* kflag = misc;                // [2 wg][2 parity]
-  volatile int* vote_kept = misc + 4;        // [VS][2]
-  int* wflag = misc + 4 + 2 * VS;            // [2 wg][2 parity][4 warps]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 4 + 2 * VS + 16);
-  volatile int* abort_flag = misc + 4 + 2 * VS + 17;
-  float* wgap = reinterpret_cast<float*>(misc + 4 + 2 * VS + 18);  // [2 wg][2 parity][4 warps]
+  // Warp vote flags [2 wg][VS][4 warps]: 1 when every row of the warp passes.
+  volatile int* wflag = misc;
+  volatile float* wgap = reinterpret_cast<volatile float*>(misc + 8 * VS);  // [2 wg][VS][4 warps]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 16 * VS);
+  volatile int* abort_flag = misc + 16 * VS + 1;
+  // First flag (and gap) of warpgroup w's vote on key tile j.
+  auto vslot = [&](int w, int j) { return (w * VS + j % VS) * 4; };
 
   const uint32_t b_qfull = smem_u32(&bars[0]);
   auto b_kfull = [&](int s) { return smem_u32(&bars[1 + s]); };
@@ -211,36 +181,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   auto b_vfull = [&](int s) { return smem_u32(&bars[1 + 2 * NK + s]); };
   auto b_vempty = [&](int s) { return smem_u32(&bars[1 + 2 * NK + NV + s]); };
   constexpr int kWgBar = 1 + 2 * NK + 2 * NV;
-  // Signals between a query tile's softmax and the MMA thread, each in two
-  // barriers taken by the parity of its index (key tile j, or kept tile k):
-  // with three S buffers a softmax step may run one tile ahead of the MMA
-  // thread's handling of the previous one, and one barrier could then
-  // complete two phases before the other side tests the first.
-  //   s_full  S(w, j) is in TMEM                 (MMA -> softmax)
-  //   vote    the decision on tile j is posted   (softmax -> MMA)
-  //   p_lo    P of the first Bc/2 keys stored    (softmax -> MMA, kept tiles)
-  //   p_hi    all of P stored                    (softmax -> MMA, kept tiles)
-  // (With one S buffer per query tile neither side can run ahead, so the
-  // first barrier of each pair serves every index.)
-  auto b_pair = [&](int base, int w, int i) {
-    return smem_u32(&bars[kWgBar + base + 2 * w + (TRIPLE ? (i & 1) : 0)]);
+  // Signals between a query tile's softmax and the MMA thread.  With one S
+  // buffer per query tile neither side can run a phase ahead of the other.
+  //   s_full  S(w, j) is in TMEM                 (MMA -> softmax; parity j)
+  //   p_lo    P of the first Bc/2 keys stored    (softmax -> MMA, kept tile k)
+  //   p_hi    all of P stored                    (softmax -> MMA, kept tile k)
+  auto b_sfull = [&](int w) { return smem_u32(&bars[kWgBar + w]); };
+  auto b_plo = [&](int w) { return smem_u32(&bars[kWgBar + 2 + w]); };
+  auto b_phi = [&](int w) { return smem_u32(&bars[kWgBar + 4 + w]); };
+  // The vote on key tile j: each softmax warp stores its flag (and gap) in
+  // slot j % VS and arrives; the MMA thread, the collector warp and the
+  // softmax warps whose own rows all passed read the four flags once the
+  // phase is complete.  vote_read: the collector has read the slot, which
+  // may then take tile j + VS.
+  auto b_vote = [&](int w, int j) { return smem_u32(&bars[kWgBar + 6 + w * VS + j % VS]); };
+  auto b_vread = [&](int w, int j) {
+    return smem_u32(&bars[kWgBar + 6 + 2 * VS + w * VS + j % VS]);
   };
-  auto pair_par = [&](int i) { return uint32_t(TRIPLE ? (i >> 1) & 1 : i & 1); };
-  auto b_sfull = [&](int w, int j) { return b_pair(0, w, j); };
-  auto b_vmma = [&](int w, int j) { return b_pair(4, w, j); };
-  auto b_plo = [&](int w, int k) { return b_pair(8, w, k); };
-  auto b_phi = [&](int w, int k) { return b_pair(12, w, k); };
-  auto b_odone = [&](int w) { return smem_u32(&bars[kWgBar + 16 + w]); }; // P.V of a kept tile done
-  auto b_vote_full = [&](int w, int s) { return smem_u32(&bars[kWgBar + 18 + w * VS + s]); };
-  auto b_vote_empty = [&](int w, int s) {
-    return smem_u32(&bars[kWgBar + 18 + 2 * VS + w * VS + s]);
-  };
-  const uint32_t b_mmadone = smem_u32(&bars[kWgBar + 18 + 4 * VS]);
-  // Turn token of a query tile's exponentials (one arrival per softmax warp).
-  auto b_tok = [&](int w) { return smem_u32(&bars[kWgBar + 19 + 4 * VS + w]); };
-  constexpr bool ALT = (TRIPLE && D == 64 && SSKIP_PF_ALT != 0) || (!TRIPLE && SSKIP_PF_ALT_D128 != 0);
-  // TMEM column of the S/P buffer of query tile w at key tile j.
-  auto s_col = [&](int w, int j) { return uint32_t((TRIPLE ? (2 * j + w) % 3 : w) * BC); };
+  auto vote_par = [&](int j) { return uint32_t((j / VS) & 1); };
+  const uint32_t b_mmadone = smem_u32(&bars[kWgBar + 6 + 4 * VS]);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -285,17 +244,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int s = 0; s < NK; ++s) { mbar_init(b_kfull(s), 1); mbar_init(b_kempty(s), 1); }
     for (int s = 0; s < NV; ++s) { mbar_init(b_vfull(s), 1); mbar_init(b_vempty(s), 1); }
     for (int w = 0; w < 2; ++w) {
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(b_sfull(w, i), 1);
-        mbar_init(b_vmma(w, i), 1);
-        mbar_init(b_plo(w, i), 4);  // one arrival per softmax warp
-        mbar_init(b_phi(w, i), 4);
-      }
-      mbar_init(b_odone(w), 1);
-      mbar_init(b_tok(w), 4);
+      mbar_init(b_sfull(w), 1);
+      mbar_init(b_plo(w), 4);  // one arrival per softmax warp
+      mbar_init(b_phi(w), 4);
     }
     for (int w = 0; w < 2; ++w)
-      for (int s = 0; s < VS; ++s) { mbar_init(b_vote_full(w, s), 1); mbar_init(b_vote_empty(w, s), 1); }
+      for (int s = 0; s < VS; ++s) { mbar_init(b_vote(w, s), 4); mbar_init(b_vread(w, s), 1); }
     mbar_init(b_mmadone, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -310,7 +264,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 4) {
-    regs_dealloc<80>();
+    regs_dealloc<SSKIP_PF_PRODUCER_REGS>();
     if (warp == 0 && lane == 0) {
       // ================= TMA producer: Q_A, Q_B, then the K ring ==========
       tma_prefetch_desc(&tmQ);
@@ -323,9 +277,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tma_load_3d(sbase + C::kQ + w * C::kQBytes + blk * 128 * 128, &tmQ, b_qfull, blk * 64,
                       row0 + 128 * w, b * p.Hq + hq);
       int last = -1;
+      const int n_w[2] = {n_a, n_b};
       for (int j = 0; j < n_j; ++j) {
         const int s = j % NK;
         if (j >= NK && !mbar_wait(b_kempty(s), ((j / NK) - 1) & 1, abort_flag)) break;
+        // No vote on tile j (which needs K_j) before the collector has read
+        // the same slots' votes on tile j - VS.
+        if (j >= VS) {
+          bool okv = true;
+#pragma unroll
+          for (int w = 0; w < 2; ++w)
+            if (okv && j - VS < n_w[w]) okv = mbar_wait(b_vread(w, j), vote_par(j) ^ 1u, abort_flag);
+          if (!okv) break;
+        }
         if (!dev_check(j < p.n_k && b * p.Hkv + kvh < p.B * p.Hkv)) {
           mbar_arrive(b_kfull(s));  // the phase completes without data
           continue;
@@ -351,11 +315,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint64_t dq0 = smem_desc_sw128(sbase + C::kQ, 16, 1024);
       const uint64_t dk0 = smem_desc_sw128(sbase + C::kK, 16, 1024);
       const uint64_t dv0 = smem_desc_sw128(sbase + C::kV, BC * 128, 1024);
-      // S = Q_w K_j^T into TMEM columns [col, col + Bc).
-      auto issue_s = [&](int w, int j, uint32_t col) {
+      // S = Q_w K_j^T into query tile w's TMEM columns [w Bc, w Bc + Bc).
+      auto issue_s = [&](int w, int j) {
         const uint64_t da = dq0 + (uint64_t)((w * C::kQBytes) >> 4);
         const uint64_t db = dk0 + (uint64_t)(((j % NK) * C::kKVBytes) >> 4);
-        const uint32_t d_tmem = tmem + col;
+        const uint32_t d_tmem = tmem + w * BC;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oa = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
@@ -364,10 +328,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
       };
       int pv_count[2] = {0, 0};
-      // O(w) += P[:, half h] V[half h], P read from TMEM columns from col, V
-      // from slot vs.
-      auto issue_pv_half = [&](int w, uint32_t col, int vs, int h) {
-        const uint32_t p_tmem = tmem + col;
+      // O(w) += P[:, half h] V[half h], P read from query tile w's S/P
+      // columns, V from slot vs.
+      auto issue_pv_half = [&](int w, int vs, int h) {
+        const uint32_t p_tmem = tmem + w * BC;
         const uint32_t o_tmem = tmem + C::kOCol + w * D;
         const uint64_t dv = dv0 + (uint64_t)((vs * C::kKVBytes) >> 4);
 #pragma unroll
@@ -379,129 +343,79 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (h == 1) ++pv_count[w];
       };
       const int n_w[2] = {n_a, n_b};
-      int kc_w[2] = {0, 0};  // kept tiles per warpgroup: index of p_lo / p_hi / o_done
+      // Whether warpgroup w keeps key tile j (some warp holds a row that did
+      // not pass); -1 when the CTA is aborting.
+      auto vote_of = [&](int w, int j) -> int {
+        if (!mbar_wait(b_vote(w, j), vote_par(j), abort_flag)) return -1;
+        const volatile int* f = wflag + vslot(w, j);
+        return (f[0] & f[1] & f[2] & f[3]) ? 0 : 1;
+      };
+      int kc_w[2] = {0, 0};  // kept tiles per warpgroup (phase of p_lo / p_hi)
       int kc = 0;            // tiles some warpgroup kept: the V load number
       bool ok = mbar_wait(b_qfull, 0, abort_flag);
-      if constexpr (!TRIPLE) {
-        // One S buffer per query tile.  Key tile j, warpgroup A then B: its
-        // decision; for a kept tile P_lo V as soon as P_lo is stored and P_hi V
-        // once P is complete; then S(j+1), which overwrites the P(j) that P.V
-        // just read.  V_j is in slot kc % NV (the V producer's numbering).
-        if (ok && n_j > 0) {
-          ok = mbar_wait(b_kfull(0), 0, abort_flag);
-          tc_fence_after();
-          if (ok) {
+      // Key tile j, warpgroup A then B: its decision; for a kept tile P_lo V
+      // as soon as P_lo is stored and P_hi V once P is complete; then S(j+1),
+      // which overwrites the P(j) that P.V just read.  V_j is in slot kc % NV
+      // (the collector's numbering).
+      if (ok && n_j > 0) {
+        ok = mbar_wait(b_kfull(0), 0, abort_flag);
+        tc_fence_after();
+        if (ok) {
 #pragma unroll
-            for (int w = 0; w < 2; ++w)
-              if (n_w[w] > 0) {
-                issue_s(w, 0, w * BC);
-                umma_commit(b_sfull(w, 0));
-              }
-            umma_commit(b_kempty(0));
-          }
-        }
-        for (int j = 0; ok && j < n_j; ++j) {
-          const int vs = kc % NV;
-          bool any_kept = false, v_ready = false, k_ready = false;
-          // K_{j+1} is waited for just before its first use, so that a late
-          // K tile never holds back a P.V.
-          auto need_k = [&]() {
-            if (!k_ready) k_ready = mbar_wait(b_kfull((j + 1) % NK), ((j + 1) / NK) & 1, abort_flag);
-            return k_ready;
-          };
-#pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            if (j >= n_w[w]) continue;
-            const bool s_next = j + 1 < n_w[w];
-            if (!mbar_wait(b_vmma(w, j), pair_par(j), abort_flag)) { ok = false; break; }
-            const bool kept = kflag[w * 2 + (j & 1)] != 0;
-            if (kept) {
-              any_kept = true;
-              const uint32_t par = pair_par(kc_w[w]);
-              if (!mbar_wait(b_plo(w, kc_w[w]), par, abort_flag)) { ok = false; break; }
-              if (!v_ready) {
-                if (!mbar_wait(b_vfull(vs), (kc / NV) & 1, abort_flag)) { ok = false; break; }
-                v_ready = true;
-              }
-              tc_fence_after();
-              issue_pv_half(w, w * BC, vs, 0);
-              if (!mbar_wait(b_phi(w, kc_w[w]), par, abort_flag)) { ok = false; break; }
-              tc_fence_after();
-              issue_pv_half(w, w * BC, vs, 1);
-              ++kc_w[w];
-              if (s_next) {
-                if (!need_k()) { ok = false; break; }
-                issue_s(w, j + 1, w * BC);
-              }
-            } else if (s_next) {
-              if (!need_k()) { ok = false; break; }
-              tc_fence_after();
-              issue_s(w, j + 1, w * BC);
+          for (int w = 0; w < 2; ++w)
+            if (n_w[w] > 0) {
+              issue_s(w, 0);
+              umma_commit(b_sfull(w));
             }
-            if (s_next) umma_commit(b_sfull(w, j + 1));
-          }
-          if (!ok) break;
-          if (any_kept) {
-            umma_commit(b_vempty(vs));
-            ++kc;
-          }
-          if (j + 1 < n_j) umma_commit(b_kempty((j + 1) % NK));
+          umma_commit(b_kempty(0));
         }
-      } else {
-        // Three S buffers.  Key tile j: A's tile j, S_B(j+1) (into the buffer
-        // A's P(j) leaves), B's tile j, S_A(j+2) (into the buffer B's P(j)
-        // leaves): each query tile's next S is ready before its softmax step
-        // ends.
-        // S(w, t) once K_t is here, then its commit.
-        auto next_s = [&](int w, int t) {
-          if (!ok || t >= n_w[w]) return;
-          ok = mbar_wait(b_kfull(t % NK), (t / NK) & 1, abort_flag);
-          if (!ok) return;
-          tc_fence_after();
-          issue_s(w, t, s_col(w, t));
-          umma_commit(b_sfull(w, t));
+      }
+      for (int j = 0; ok && j < n_j; ++j) {
+        const int vs = kc % NV;
+        bool any_kept = false, v_ready = false, k_ready = false;
+        // K_{j+1} is waited for just before its first use, so that a late
+        // K tile never holds back a P.V.
+        auto need_k = [&]() {
+          if (!k_ready) k_ready = mbar_wait(b_kfull((j + 1) % NK), ((j + 1) / NK) & 1, abort_flag);
+          return k_ready;
         };
-        bool any_kept = false, v_ready = false;
-        // Warpgroup w's tile j: its decision; for a kept tile P_lo V as soon
-        // as P_lo is stored and P_hi V once P is complete, then o_done.
-        auto process = [&](int w, int j, int vs) {
-          if (!ok || j >= n_w[w]) return;
-          if (!(ok = mbar_wait(b_vmma(w, j), pair_par(j), abort_flag))) return;
-          if (!kflag[w * 2 + (j & 1)]) return;
-          any_kept = true;
-          const int k = kc_w[w];
-          if (!(ok = mbar_wait(b_plo(w, k), pair_par(k), abort_flag))) return;
-          if (!v_ready) {
-            if (!(ok = mbar_wait(b_vfull(vs), (kc / NV) & 1, abort_flag))) return;
-            v_ready = true;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          if (j >= n_w[w]) continue;
+          const bool s_next = j + 1 < n_w[w];
+          const int kv = vote_of(w, j);
+          if (kv < 0) { ok = false; break; }
+          if (kv) {
+            any_kept = true;
+            const uint32_t par = kc_w[w] & 1;
+            if (!mbar_wait(b_plo(w), par, abort_flag)) { ok = false; break; }
+            if (!v_ready) {
+              if (!mbar_wait(b_vfull(vs), (kc / NV) & 1, abort_flag)) { ok = false; break; }
+              v_ready = true;
+            }
+            tc_fence_after();
+            issue_pv_half(w, vs, 0);
+            if (!mbar_wait(b_phi(w), par, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv_half(w, vs, 1);
+            ++kc_w[w];
+            if (s_next) {
+              if (!need_k()) { ok = false; break; }
+              issue_s(w, j + 1);
+            }
+          } else if (s_next) {
+            if (!need_k()) { ok = false; break; }
+            tc_fence_after();
+            issue_s(w, j + 1);
           }
-          tc_fence_after();
-          issue_pv_half(w, s_col(w, j), vs, 0);
-          if (!(ok = mbar_wait(b_phi(w, k), pair_par(k), abort_flag))) return;
-          tc_fence_after();
-          issue_pv_half(w, s_col(w, j), vs, 1);
-          umma_commit(b_odone(w));
-          ++kc_w[w];
-        };
-        next_s(0, 0);
-        next_s(1, 0);
-        next_s(0, 1);
-        if (ok && n_j > 0) umma_commit(b_kempty(0));
-        for (int j = 0; ok && j < n_j; ++j) {
-          const int vs = kc % NV;
-          any_kept = false;
-          v_ready = false;
-          process(0, j, vs);
-          next_s(1, j + 1);
-          process(1, j, vs);
-          next_s(0, j + 2);
-          if (!ok) break;
-          if (any_kept) {
-            umma_commit(b_vempty(vs));
-            ++kc;
-          }
-          if (j + 1 < n_j) umma_commit(b_kempty((j + 1) % NK));
+          if (s_next) umma_commit(b_sfull(w));
         }
+        if (!ok) break;
+        if (any_kept) {
+          umma_commit(b_vempty(vs));
+          ++kc;
+        }
+        if (j + 1 < n_j) umma_commit(b_kempty((j + 1) % NK));
       }
       // Every MMA issued by this thread completes before the epilogue reads O
       // and before TMEM is released.
@@ -509,33 +423,62 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       int no_abort = 0;
       mbar_wait(b_mmadone, 0, &no_abort);
     } else if (warp == 2 && lane == 0) {
-      // ================= V producer: issues V_j on the FIRST keep vote =====
-      // Each warpgroup posts its vote on tile j as soon as it has its row
-      // maxima; the first "keep" starts the V_j load, so its latency hides
-      // behind that warpgroup's exponentials.  Loads are numbered in tile
-      // order over the tiles some warpgroup kept and go to slot number % NV;
-      // a tile both skip costs nothing here.  Both votes are consumed in order
-      // to keep the vote slots' phases exact.
+      // ================= collector: reads the votes, issues V, records =====
+      // Both query tiles' votes on tile j, in tile order.  The first "keep"
+      // starts the V_j load, so its latency hides behind that warpgroup's
+      // exponentials.  Loads are numbered in tile order over the tiles some
+      // warpgroup kept and go to slot number % NV; a tile both skip costs
+      // nothing here.  The tile records and the counts are written here too,
+      // off the softmax warps' path.
       tma_prefetch_desc(&tmV);
+      const int n_w[2] = {n_a, n_b};
       int kc = 0, last = -1;
+      long long n_vis = 0, n_skip = 0;
       for (int j = 0; j < n_j && !*abort_flag; ++j) {
-        const int vslot = j % VS;
-        const uint32_t par = (j / VS) & 1;
-        bool seen[2] = {false, false}, kept_any = false, issued = false;
-        const uint64_t t0 = globaltimer_ns();
-        while (!(seen[0] && seen[1])) {
-          bool progress = false;
+        bool issued = false;
 #pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            if (!seen[w] && mbar_test_wait(b_vote_full(w, vslot), par)) {
-              seen[w] = true;
-              progress = true;
-              kept_any = kept_any || vote_kept[vslot * 2 + w] != 0;
-              mbar_arrive(b_vote_empty(w, vslot));
-            }
+        for (int w = 0; w < 2; ++w) {
+          if (j >= n_w[w]) continue;
+          if (!mbar_wait(b_vote(w, j), vote_par(j), abort_flag)) break;
+          const int fs = vslot(w, j);
+          int fl[4];
+          float gm[NGRP];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) fl[q] = wflag[fs + q];
+#pragma unroll
+          for (int g = 0; g < NGRP; ++g) {
+            gm[g] = -INFINITY;
+            if (EXT && p.tile_crit)
+#pragma unroll
+              for (int q = 0; q < WPG; ++q) gm[g] = fmaxf(gm[g], wgap[fs + g * WPG + q]);
           }
-          if (!progress) __nanosleep(40);  // leave issue slots to the softmax warps
-          if (kept_any && !issued) {
+          mbar_arrive(b_vread(w, j));  // the slot may now take tile j + VS
+          bool kept = false;
+#pragma unroll
+          for (int g = 0; g < NGRP; ++g) {
+            bool all = true;
+            uint32_t bits = 0;
+#pragma unroll
+            for (int q = 0; q < WPG; ++q) {
+              all = all && fl[g * WPG + q] != 0;
+              bits |= fl[g * WPG + q] != 0 ? (1u << q) : 0u;
+            }
+            const int it = (row0 + 128 * w) / BR + g;  // this group's query tile
+            if (it >= p.n_q) continue;
+            const int jm = CAUSAL ? min(p.n_k - 1, ((it + 1) * BR - 1) / BC) : p.n_k - 1;
+            if (j > jm) continue;  // the group does not visit tile j
+            kept = kept || !all;
+            const size_t rec = (((size_t)b * p.Hq + hq) * p.n_q + it) * p.n_k + j;
+            if (!dev_check(j < p.n_k && rec < (size_t)p.B * p.Hq * p.n_q * p.n_k)) continue;
+            ++n_vis;
+            n_skip += all ? 1 : 0;
+            if (p.tile_state) p.tile_state[rec] = all ? 2 : 1;
+            if (EXT && p.slice_mask)
+              p.slice_mask[rec] = uint8_t(0x80u | (p.slice_vote ? bits : (all ? 1u : 0u)));
+            // Skipped iff ln(tsf) > max gap * ln 2 + ln L (for every factor below L).
+            if (EXT && p.tile_crit) p.tile_crit[rec] = gm[g] * 0.69314718055994531f + p.ln_L;
+          }
+          if (kept && !issued) {
             const int vs = kc % NV;
             if (kc >= NV && !mbar_wait(b_vempty(vs), ((kc / NV) - 1) & 1, abort_flag)) break;
             if (!dev_check(j < p.n_k && vs < NV)) {
@@ -550,18 +493,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             issued = true;
             last = kc++;
           }
-          if (*abort_flag) break;
-          if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            latch_status(kStatusTimeout);
-            break;
-          }
         }
       }
       if (*abort_flag) {
         int dummy = 0;
         for (int k = max(0, last - NV + 1); k <= last; ++k)
           mbar_wait(b_vfull(k % NV), (k / NV) & 1, &dummy);
+      }
+      if (p.counts) {
+        atomicAdd(&p.counts[0], (unsigned long long)n_skip);
+        atomicAdd(&p.counts[1], (unsigned long long)n_vis);
+        if (EXT && p.n_counts == 4 && !p.slice_vote) {  // one slice per block
+          atomicAdd(&p.counts[2], (unsigned long long)n_skip);
+          atomicAdd(&p.counts[3], (unsigned long long)n_vis);
+        }
       }
     }
   } else {
@@ -575,18 +520,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const bool row_in = row < p.L;
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
     const uint32_t tO = tmem + C::kOCol + wg * D + lane_base;
-    int n_kept = 0;  // kept tiles of this query tile so far (parity of o_done)
     const int n_own = wg == 0 ? n_a : n_b;
-    int g_tile[NGRP], g_jmax[NGRP];
-#pragma unroll
-    for (int g = 0; g < NGRP; ++g) {
-      g_tile[g] = (row0 + 128 * wg) / BR + g;
-      const int jm = CAUSAL ? min(p.n_k - 1, ((g_tile[g] + 1) * BR - 1) / BC) : p.n_k - 1;
-      g_jmax[g] = g_tile[g] < p.n_q ? jm : -1;
-    }
-    const int my_jmax = g_jmax[grp];
-    const bool elected = (wq == 0 && lane == 0);
-    const int bar_id = 1 + wg;
+    // Last key tile this row's vote group visits (-1: the group is padding).
+    const int my_tile = (row0 + 128 * wg) / BR + grp;
+    const int my_jmax = my_tile >= p.n_q ? -1
+                        : CAUSAL ? min(p.n_k - 1, ((my_tile + 1) * BR - 1) / BC) : p.n_k - 1;
     const float log2_t = p.log2_t;
     const bool t_pos = p.t_positive != 0;
     const float scale = p.scale_log2;
@@ -594,14 +532,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // l_run sums P in fp32 (for lse); lr_run sums the bf16-rounded P that the
     // P.V MMA applied, so that O / lr_run weighs V with weights summing to 1.
     float m_run = -INFINITY, m_ref = -INFINITY, l_run = 0.f, lr_run = 0.f;
-    long long n_vis = 0, n_skip = 0, n_svis = 0, n_sskip = 0;
+    long long n_svis = 0, n_sskip = 0;
 
-    auto post_vote = [&](int j, bool kept) {  // elected thread only
-      const int vslot = j % VS;
-      if (j >= VS) mbar_wait(b_vote_empty(wg, vslot), ((j / VS) - 1) & 1, abort_flag);
-      vote_kept[vslot * 2 + wg] = kept ? 1 : 0;
-      mbar_arrive(b_vote_full(wg, vslot));
-    };
     // This warp's part of a signal counted once per softmax warp: its TMEM
     // accesses are complete (the caller waited for them) and ordered before
     // the MMA warp's next tcgen05 operation.
@@ -610,30 +542,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar);
     };
-
-    // Turns (ALT): the exponentials of A's tile j follow B's of tile j - 1,
-    // B's of tile j follow A's of tile j; a tile without exponentials passes
-    // its turn at once.  Each warp waits for the other query tile's four
-    // warps and hands its own turn on.
-    auto take_turn = [&](int j) {
-      if (ALT && (wg == 1 || j > 0))
-        mbar_wait(b_tok(1 - wg), (wg == 1 ? j : j - 1) & 1, abort_flag);
-    };
-    auto pass_turn = [&]() {
-      if (ALT) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(b_tok(wg));
-      }
-    };
     for (int j = 0; j < n_j; ++j) {
-      if (j >= n_own) {  // this tile has no row here: vote "not kept" only
-        if (elected) post_vote(j, false);
-        take_turn(j);
-        pass_turn();
-        continue;
-      }
-      const uint32_t tS = tmem + s_col(wg, j) + lane_base;
-      mbar_wait(b_sfull(wg, j), pair_par(j), abort_flag);
+      if (j >= n_own) break;  // no row of this query tile visits tile j or later
+      const uint32_t tS = tmem + wg * BC + lane_base;
+      mbar_wait(b_sfull(wg), j & 1, abort_flag);
       tc_fence_after();
       __syncwarp();
       uint32_t sr[BC];
@@ -665,72 +577,47 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const bool gvis = j <= my_jmax;
       const bool pass = row_passes_log2(m_loc, m_run, log2_t, t_pos);
       const bool wall = __all_sync(0xffffffffu, !(row_in && gvis) || pass);
-      if (lane == 0) wflag[(wg * 2 + (j & 1)) * 4 + wq] = wall ? 1 : 0;
+      const int fs = vslot(wg, j);
       if (EXT && p.tile_crit) {
         // Largest gap m_local - m_run over the warp's valid rows (log2 units).
         float gap = (!(row_in && gvis) || m_loc == -INFINITY) ? -INFINITY
                     : (m_run == -INFINITY) ? INFINITY : m_loc - m_run;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) gap = fmaxf(gap, __shfl_xor_sync(0xffffffffu, gap, o));
-        if (lane == 0) wgap[(wg * 2 + (j & 1)) * 4 + wq] = gap;
+        if (lane == 0) wgap[fs + wq] = gap;
       }
-      // Every warp's S loads are complete before this barrier, so after it
-      // the whole S(j) has been read once.
+      // This warp's loads of S(j) are complete: once all four warps have
+      // arrived, the MMA thread may reuse the columns.
       tc_fence_before();
-      named_bar_sync(bar_id, 128);
-      bool g_kept[NGRP];
-      bool tile_kept = false;
+      __syncwarp();
+      if (lane == 0) {
+        wflag[fs + wq] = wall ? 1 : 0;
+        mbar_arrive(b_vote(wg, j));
+      }
+      // A warp holding a row that did not pass knows at once that its group,
+      // and so the tile, is kept.  A warp whose rows all passed reads the
+      // other warps' flags.
+      bool grp_kept = true, tile_kept = true;
+      if (wall) {
+        mbar_wait(b_vote(wg, j), vote_par(j), abort_flag);
+        int fl[4];
 #pragma unroll
-      for (int g = 0; g < NGRP; ++g) {
-        bool all = true;
-        uint32_t bits = 0;
+        for (int q = 0; q < 4; ++q) fl[q] = wflag[fs + q];
+        tile_kept = !(fl[0] & fl[1] & fl[2] & fl[3]);
+        grp_kept = false;
 #pragma unroll
-        for (int w = 0; w < WPG; ++w) {
-          const bool f = wflag[(wg * 2 + (j & 1)) * 4 + g * WPG + w] != 0;
-          all = all && f;
-          bits |= f ? (1u << w) : 0u;
-        }
-        const bool vis = j <= g_jmax[g];
-        g_kept[g] = vis && !all;
-        tile_kept = tile_kept || g_kept[g];
-        if (elected && vis) {
-          const size_t rec = (((size_t)b * p.Hq + hq) * p.n_q + g_tile[g]) * p.n_k + j;
-          if (!dev_check(g_tile[g] < p.n_q && j < p.n_k &&
-                         rec < (size_t)p.B * p.Hq * p.n_q * p.n_k))
-            continue;
-          ++n_vis;
-          n_skip += all ? 1 : 0;
-          if (p.tile_state) p.tile_state[rec] = all ? 2 : 1;
-          if (EXT && p.slice_mask)
-            p.slice_mask[rec] = uint8_t(0x80u | (p.slice_vote ? bits : (all ? 1u : 0u)));
-          if (EXT && p.tile_crit) {
-            // Skipped iff ln(tsf) > max gap * ln 2 + ln L (for every factor below L).
-            float gm = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < WPG; ++w) gm = fmaxf(gm, wgap[(wg * 2 + (j & 1)) * 4 + g * WPG + w]);
-            p.tile_crit[rec] = gm * 0.69314718055994531f + p.ln_L;
-          }
-        }
+        for (int q = 0; q < WPG; ++q) grp_kept = grp_kept || fl[grp * WPG + q] == 0;
       }
       // Slice counters: warps holding at least one valid row of a visiting group.
       if (EXT && lane == 0 && gvis && row0 + 128 * wg + wq * 32 < p.L) {
         ++n_svis;
         n_sskip += wall ? 1 : 0;
       }
-      if (elected) {
-        post_vote(j, tile_kept);
-        kflag[wg * 2 + (j & 1)] = tile_kept ? 1 : 0;
-        mbar_arrive(b_vmma(wg, j));
-      }
-      if (!tile_kept) {
-        take_turn(j);
-        pass_turn();
-        continue;
-      }
+      if (!tile_kept) continue;
 
       // Block vote: every row of a kept group updates.  Warp vote: only the
       // rows of a warp slice that did not pass.
-      const bool mine = row_in && ((EXT && p.slice_vote) ? (gvis && !wall) : g_kept[grp]);
+      const bool mine = row_in && ((EXT && p.slice_vote) ? (gvis && !wall) : grp_kept);
       float alpha = 1.f;
       bool rescale = false;
       if (mine) {
@@ -752,14 +639,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint64_t nref2 = f2pack(nref, nref);
       __syncwarp();
       if (__any_sync(0xffffffffu, rescale)) {
-        // O must hold every earlier P.V.  With one S buffer per query tile it
-        // does: S(j) was committed after P.V(j-1).  With three, S(j) may be
-        // ready first, so wait for the last kept tile's P.V (a rescale needs
-        // an earlier kept tile, so n_kept >= 1).
-        if (TRIPLE) {
-          mbar_wait(b_odone(wg), (n_kept - 1) & 1, abort_flag);
-          tc_fence_after();
-        }
+        // O holds every earlier P.V: S(j) was committed after P.V(j-1).
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float o32[32];
@@ -806,16 +686,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         else tmem_st16(tS + h * HP, pk);
       };
       if (none) {
-        take_turn(j);
-        pass_turn();
 #pragma unroll
         for (int i = 0; i < HP; ++i) pk[i] = 0u;
         store_half(0);
         tmem_st_wait();
-        warp_signal(b_plo(wg, n_kept));
+        warp_signal(b_plo(wg));
         store_half(1);
         tmem_st_wait();
-        warp_signal(b_phi(wg, n_kept));
+        warp_signal(b_phi(wg));
       } else if constexpr (kReload<D>() || (EXT && SSKIP_PF_EXT_RELOAD)) {
         // The row max is known; re-read each half of S (its columns are still
         // intact: P of the first half lands in the first quarter).  The second
@@ -837,33 +715,28 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         };
         load_half(0);
-        take_turn(j);
         wait_half(0);
         exp_half(0, reinterpret_cast<const float*>(rr));
         store_half(0);
         load_half(1);
         tmem_st_wait();
-        warp_signal(b_plo(wg, n_kept));
+        warp_signal(b_plo(wg));
         wait_half(1);
         exp_half(1, reinterpret_cast<const float*>(rr));
-        pass_turn();
         store_half(1);
         tmem_st_wait();
-        warp_signal(b_phi(wg, n_kept));
+        warp_signal(b_phi(wg));
       } else {
         // S stays in registers from the max pass (already masked).
-        take_turn(j);
         exp_half(0, s);
         store_half(0);
         tmem_st_wait();
-        warp_signal(b_plo(wg, n_kept));
+        warp_signal(b_plo(wg));
         exp_half(1, s + HK);
-        pass_turn();
         store_half(1);
         tmem_st_wait();
-        warp_signal(b_phi(wg, n_kept));
+        warp_signal(b_phi(wg));
       }
-      ++n_kept;
       if (!none) {
         uint64_t sum2 = sum2v[0], sumr2 = sumr2v[0];
 #pragma unroll
@@ -907,14 +780,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (store)
       p.lse[((size_t)b * p.Hq + hq) * p.L + row] =
           (m_ref - kPackBias + __log2f(l_run)) * 0.69314718055994531f;
-    if (elected && p.counts) {
-      atomicAdd(&p.counts[0], (unsigned long long)n_skip);
-      atomicAdd(&p.counts[1], (unsigned long long)n_vis);
-      if (EXT && p.n_counts == 4 && !p.slice_vote) {  // one slice per block
-        atomicAdd(&p.counts[2], (unsigned long long)n_skip);
-        atomicAdd(&p.counts[3], (unsigned long long)n_vis);
-      }
-    }
     if (EXT && lane == 0 && p.counts && p.n_counts == 4 && p.slice_vote && n_svis > 0) {
       atomicAdd(&p.counts[2], (unsigned long long)n_sskip);
       atomicAdd(&p.counts[3], (unsigned long long)n_svis);

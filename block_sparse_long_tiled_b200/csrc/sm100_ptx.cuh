@@ -80,37 +80,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test of the phase with the given parity.
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Non-blocking test of two barriers at once (both tests in flight together):
-// bit 0 set when bar0's phase with parity par0 is complete, bit 1 for bar1.
-__device__ __forceinline__ uint32_t mbar_test_wait2(uint32_t bar0, uint32_t par0, uint32_t bar1,
-                                                    uint32_t par1) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred q0, q1;\n\t.reg .u32 t0, t1;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 q0, [%1], %2;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 q1, [%3], %4;\n\t"
-      "selp.u32 t0, 1, 0, q0;\n\t"
-      "selp.u32 t1, 2, 0, q1;\n\t"
-      "or.b32 %0, t0, t1;\n\t}\n"
-      : "=r"(r)
-      : "r"(bar0), "r"(par0), "r"(bar1), "r"(par1)
-      : "memory");
-  return r;
-}
-
 // Bounded wait for the phase with the given parity. Returns false when the CTA
 // is aborting (another role gave up) or when this wait itself ran out.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
