@@ -95,6 +95,18 @@ __device__ __forceinline__ constexpr bool kReload() {
 #ifndef SSKIP_PF_PRODUCER_REGS
 #define SSKIP_PF_PRODUCER_REGS 88  // registers of the producer, MMA and collector warps (<= 88 with 208)
 #endif
+#ifndef SSKIP_PF_MAXACC
+#define SSKIP_PF_MAXACC 4       // independent accumulators of the row max (4 or 8)
+#endif
+#ifndef SSKIP_PF_KEEP_HALF0
+#define SSKIP_PF_KEEP_HALF0 1   // re-read path: the first half's exponentials use the max pass's registers
+#endif
+#ifndef SSKIP_PF_EARLY_LOAD1
+#define SSKIP_PF_EARLY_LOAD1 0  // with KEEP_HALF0: the second half's load is issued before the first half's exponentials
+#endif
+#ifndef SSKIP_PF_PLO_ALL
+#define SSKIP_PF_PLO_ALL 1      // every visited tile arrives on p_lo (a skipped one at its decision)
+#endif
 #ifndef SSKIP_PF_FMA_EXP_D64
 #define SSKIP_PF_FMA_EXP_D64 SSKIP_PF_FMA_EXP  // the same, for head dim 64
 #endif
@@ -383,12 +395,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int w = 0; w < 2; ++w) {
           if (j >= n_w[w]) continue;
           const bool s_next = j + 1 < n_w[w];
-          const int kv = vote_of(w, j);
+          int kv;
+          if (SSKIP_PF_PLO_ALL) {
+            // p_lo of every visited tile: the flags are stored before it.
+            if (!mbar_wait(b_plo(w), j & 1, abort_flag)) { ok = false; break; }
+            const volatile int* f = wflag + vslot(w, j);
+            kv = (f[0] & f[1] & f[2] & f[3]) ? 0 : 1;
+          } else {
+            kv = vote_of(w, j);
+          }
           if (kv < 0) { ok = false; break; }
           if (kv) {
             any_kept = true;
             const uint32_t par = kc_w[w] & 1;
-            if (!mbar_wait(b_plo(w), par, abort_flag)) { ok = false; break; }
+            if (!SSKIP_PF_PLO_ALL && !mbar_wait(b_plo(w), par, abort_flag)) { ok = false; break; }
             if (!v_ready) {
               if (!mbar_wait(b_vfull(vs), (kc / NV) & 1, abort_flag)) { ok = false; break; }
               v_ready = true;
@@ -565,15 +585,28 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (key >= p.L || (CAUSAL && key > row)) s[c] = -INFINITY;
         }
       }
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+      float m_loc;
+      if constexpr (SSKIP_PF_MAXACC == 8) {
+        float mx[8];
 #pragma unroll
-      for (int c = 0; c < BC; c += 8) {
-        mx0 = fmax3(mx0, s[c], s[c + 1]);
-        mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
-        mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
-        mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
+        for (int a = 0; a < 8; ++a) mx[a] = fmaxf(s[2 * a], s[2 * a + 1]);
+#pragma unroll
+        for (int c = 16; c < BC; c += 16)
+#pragma unroll
+          for (int a = 0; a < 8; ++a) mx[a] = fmax3(mx[a], s[c + 2 * a], s[c + 2 * a + 1]);
+        m_loc = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+      } else {
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BC; c += 8) {
+          mx0 = fmax3(mx0, s[c], s[c + 1]);
+          mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+          mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+          mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
+        }
+        m_loc = fmax3(mx0, mx1, fmaxf(mx2, mx3));
       }
-      const float m_loc = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * scale;  // scale > 0
+      m_loc *= scale;  // scale > 0
       const bool gvis = j <= my_jmax;
       const bool pass = row_passes_log2(m_loc, m_run, log2_t, t_pos);
       const bool wall = __all_sync(0xffffffffu, !(row_in && gvis) || pass);
@@ -613,7 +646,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         ++n_svis;
         n_sskip += wall ? 1 : 0;
       }
-      if (!tile_kept) continue;
+      if (!tile_kept) {
+        if (SSKIP_PF_PLO_ALL) warp_signal(b_plo(wg));
+        continue;
+      }
 
       // Block vote: every row of a kept group updates.  Warp vote: only the
       // rows of a warp slice that did not pass.
@@ -714,11 +750,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             }
           }
         };
-        load_half(0);
-        wait_half(0);
-        exp_half(0, reinterpret_cast<const float*>(rr));
+        if (SSKIP_PF_KEEP_HALF0) {
+          if (SSKIP_PF_EARLY_LOAD1) load_half(1);
+          exp_half(0, s);  // the max pass's registers (already masked)
+        } else {
+          load_half(0);
+          wait_half(0);
+          exp_half(0, reinterpret_cast<const float*>(rr));
+        }
         store_half(0);
-        load_half(1);
+        if (!(SSKIP_PF_KEEP_HALF0 && SSKIP_PF_EARLY_LOAD1)) load_half(1);
         tmem_st_wait();
         warp_signal(b_plo(wg));
         wait_half(1);
