@@ -90,7 +90,7 @@ __device__ __forceinline__ constexpr bool kReload() {
 #define SSKIP_PF_ROUNDED_L 0  // 1: O is divided by the sum of the bf16 P that P.V used
 #endif
 #ifndef SSKIP_PF_EXT_RELOAD
-#define SSKIP_PF_EXT_RELOAD 1  // the per-warp-vote build re-reads S at every d
+#define SSKIP_PF_EXT_RELOAD 0  // 1: the per-warp-vote build re-reads S at every d
 #endif
 #ifndef SSKIP_PF_PRODUCER_REGS
 #define SSKIP_PF_PRODUCER_REGS 88  // registers of the producer, MMA and collector warps (<= 88 with 208)
