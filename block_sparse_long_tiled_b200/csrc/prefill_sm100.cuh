@@ -74,7 +74,7 @@ constexpr int kPfVoteSlots = 4;
 #define SSKIP_PF_FMA_EXP 0   // element pairs per 8 whose exp2 runs on the FMA pipe
 #endif
 #ifndef SSKIP_PF_RELOAD
-#define SSKIP_PF_RELOAD 1     // re-read S from TMEM in halves for the exponentials (d = 128)
+#define SSKIP_PF_RELOAD 1     // d = 128: re-read S's second half from TMEM for the exponentials (0: hold all of S)
 #endif
 #ifndef SSKIP_PF_RELOAD_D64
 #define SSKIP_PF_RELOAD_D64 0  // at d = 64 S stays in registers from the max pass
@@ -94,18 +94,6 @@ __device__ __forceinline__ constexpr bool kReload() {
 #endif
 #ifndef SSKIP_PF_PRODUCER_REGS
 #define SSKIP_PF_PRODUCER_REGS 88  // registers of the producer, MMA and collector warps (<= 88 with 208)
-#endif
-#ifndef SSKIP_PF_MAXACC
-#define SSKIP_PF_MAXACC 4       // independent accumulators of the row max (4 or 8)
-#endif
-#ifndef SSKIP_PF_KEEP_HALF0
-#define SSKIP_PF_KEEP_HALF0 1   // re-read path: the first half's exponentials use the max pass's registers
-#endif
-#ifndef SSKIP_PF_EARLY_LOAD1
-#define SSKIP_PF_EARLY_LOAD1 0  // with KEEP_HALF0: the second half's load is issued before the first half's exponentials
-#endif
-#ifndef SSKIP_PF_PLO_ALL
-#define SSKIP_PF_PLO_ALL 1      // every visited tile arrives on p_lo (a skipped one at its decision)
 #endif
 #ifndef SSKIP_PF_FMA_EXP_D64
 #define SSKIP_PF_FMA_EXP_D64 SSKIP_PF_FMA_EXP  // the same, for head dim 64
@@ -196,16 +184,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   // Signals between a query tile's softmax and the MMA thread.  With one S
   // buffer per query tile neither side can run a phase ahead of the other.
   //   s_full  S(w, j) is in TMEM                 (MMA -> softmax; parity j)
-  //   p_lo    P of the first Bc/2 keys stored    (softmax -> MMA, kept tile k)
+  //   p_lo    P of the first Bc/2 keys stored, or the tile skipped
+  //                                              (softmax -> MMA; parity j)
   //   p_hi    all of P stored                    (softmax -> MMA, kept tile k)
   auto b_sfull = [&](int w) { return smem_u32(&bars[kWgBar + w]); };
   auto b_plo = [&](int w) { return smem_u32(&bars[kWgBar + 2 + w]); };
   auto b_phi = [&](int w) { return smem_u32(&bars[kWgBar + 4 + w]); };
   // The vote on key tile j: each softmax warp stores its flag (and gap) in
-  // slot j % VS and arrives; the MMA thread, the collector warp and the
-  // softmax warps whose own rows all passed read the four flags once the
-  // phase is complete.  vote_read: the collector has read the slot, which
-  // may then take tile j + VS.
+  // slot j % VS and arrives; the collector warp and the softmax warps whose
+  // own rows all passed read the four flags once the phase is complete (the
+  // MMA thread reads them after p_lo).  vote_read: the collector has read the
+  // slot, which may then take tile j + VS.
   auto b_vote = [&](int w, int j) { return smem_u32(&bars[kWgBar + 6 + w * VS + j % VS]); };
   auto b_vread = [&](int w, int j) {
     return smem_u32(&bars[kWgBar + 6 + 2 * VS + w * VS + j % VS]);
@@ -355,13 +344,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (h == 1) ++pv_count[w];
       };
       const int n_w[2] = {n_a, n_b};
-      // Whether warpgroup w keeps key tile j (some warp holds a row that did
-      // not pass); -1 when the CTA is aborting.
-      auto vote_of = [&](int w, int j) -> int {
-        if (!mbar_wait(b_vote(w, j), vote_par(j), abort_flag)) return -1;
-        const volatile int* f = wflag + vslot(w, j);
-        return (f[0] & f[1] & f[2] & f[3]) ? 0 : 1;
-      };
       int kc_w[2] = {0, 0};  // kept tiles per warpgroup (phase of p_lo / p_hi)
       int kc = 0;            // tiles some warpgroup kept: the V load number
       bool ok = mbar_wait(b_qfull, 0, abort_flag);
@@ -395,20 +377,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int w = 0; w < 2; ++w) {
           if (j >= n_w[w]) continue;
           const bool s_next = j + 1 < n_w[w];
-          int kv;
-          if (SSKIP_PF_PLO_ALL) {
-            // p_lo of every visited tile: the flags are stored before it.
-            if (!mbar_wait(b_plo(w), j & 1, abort_flag)) { ok = false; break; }
-            const volatile int* f = wflag + vslot(w, j);
-            kv = (f[0] & f[1] & f[2] & f[3]) ? 0 : 1;
-          } else {
-            kv = vote_of(w, j);
-          }
-          if (kv < 0) { ok = false; break; }
-          if (kv) {
+          // Every visited tile completes one p_lo phase (a skipped one at its
+          // decision); the four flags are stored before it.
+          if (!mbar_wait(b_plo(w), j & 1, abort_flag)) { ok = false; break; }
+          const volatile int* f = wflag + vslot(w, j);
+          if (!(f[0] & f[1] & f[2] & f[3])) {
             any_kept = true;
             const uint32_t par = kc_w[w] & 1;
-            if (!SSKIP_PF_PLO_ALL && !mbar_wait(b_plo(w), par, abort_flag)) { ok = false; break; }
             if (!v_ready) {
               if (!mbar_wait(b_vfull(vs), (kc / NV) & 1, abort_flag)) { ok = false; break; }
               v_ready = true;
@@ -585,28 +560,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (key >= p.L || (CAUSAL && key > row)) s[c] = -INFINITY;
         }
       }
-      float m_loc;
-      if constexpr (SSKIP_PF_MAXACC == 8) {
-        float mx[8];
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int a = 0; a < 8; ++a) mx[a] = fmaxf(s[2 * a], s[2 * a + 1]);
-#pragma unroll
-        for (int c = 16; c < BC; c += 16)
-#pragma unroll
-          for (int a = 0; a < 8; ++a) mx[a] = fmax3(mx[a], s[c + 2 * a], s[c + 2 * a + 1]);
-        m_loc = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-      } else {
-        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < BC; c += 8) {
-          mx0 = fmax3(mx0, s[c], s[c + 1]);
-          mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
-          mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
-          mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
-        }
-        m_loc = fmax3(mx0, mx1, fmaxf(mx2, mx3));
+      for (int c = 0; c < BC; c += 8) {
+        mx0 = fmax3(mx0, s[c], s[c + 1]);
+        mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+        mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+        mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
       }
-      m_loc *= scale;  // scale > 0
+      const float m_loc = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * scale;  // scale > 0
       const bool gvis = j <= my_jmax;
       const bool pass = row_passes_log2(m_loc, m_run, log2_t, t_pos);
       const bool wall = __all_sync(0xffffffffu, !(row_in && gvis) || pass);
@@ -647,7 +609,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         n_sskip += wall ? 1 : 0;
       }
       if (!tile_kept) {
-        if (SSKIP_PF_PLO_ALL) warp_signal(b_plo(wg));
+        warp_signal(b_plo(wg));  // the MMA thread's signal that tile j is skipped
         continue;
       }
 
@@ -731,38 +693,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tmem_st_wait();
         warp_signal(b_phi(wg));
       } else if constexpr (kReload<D>() || (EXT && SSKIP_PF_EXT_RELOAD)) {
-        // The row max is known; re-read each half of S (its columns are still
-        // intact: P of the first half lands in the first quarter).  The second
-        // half's load is in flight while P_lo lands.
+        // The first half's exponentials use the max pass's registers (already
+        // masked); the second half of S is re-read from TMEM (its columns are
+        // intact: P of the first half lands in the first quarter), its load in
+        // flight while P_lo lands.  Only 64 registers of S stay live past the
+        // max pass.
         uint32_t rr[HK];
-        auto load_half = [&](int h) {
-          tmem_ld32_async(tS + h * HK, rr);
-          if constexpr (HK == 64) tmem_ld32_async(tS + h * HK + 32, rr + 32);
-        };
-        auto wait_half = [&](int h) {
-          if constexpr (HK == 64) tmem_wait_ld_tie64(rr);
-          else tmem_wait_ld_tie32(rr);
-          if (need_mask) {
-#pragma unroll
-            for (int c = 0; c < HK; ++c) {
-              const int key = key0 + h * HK + c;
-              if (key >= p.L || (CAUSAL && key > row)) rr[c] = __float_as_uint(-INFINITY);
-            }
-          }
-        };
-        if (SSKIP_PF_KEEP_HALF0) {
-          if (SSKIP_PF_EARLY_LOAD1) load_half(1);
-          exp_half(0, s);  // the max pass's registers (already masked)
-        } else {
-          load_half(0);
-          wait_half(0);
-          exp_half(0, reinterpret_cast<const float*>(rr));
-        }
+        exp_half(0, s);
         store_half(0);
-        if (!(SSKIP_PF_KEEP_HALF0 && SSKIP_PF_EARLY_LOAD1)) load_half(1);
+        tmem_ld32_async(tS + HK, rr);
+        if constexpr (HK == 64) tmem_ld32_async(tS + HK + 32, rr + 32);
         tmem_st_wait();
         warp_signal(b_plo(wg));
-        wait_half(1);
+        if constexpr (HK == 64) tmem_wait_ld_tie64(rr);
+        else tmem_wait_ld_tie32(rr);
+        if (need_mask) {
+#pragma unroll
+          for (int c = 0; c < HK; ++c) {
+            const int key = key0 + HK + c;
+            if (key >= p.L || (CAUSAL && key > row)) rr[c] = __float_as_uint(-INFINITY);
+          }
+        }
         exp_half(1, reinterpret_cast<const float*>(rr));
         store_half(1);
         tmem_st_wait();
