@@ -74,7 +74,7 @@ constexpr int kPfVoteSlots = 4;
 #define SSKIP_PF_FMA_EXP 0   // element pairs per 8 whose exp2 runs on the FMA pipe
 #endif
 #ifndef SSKIP_PF_RELOAD
-#define SSKIP_PF_RELOAD 1     // d = 128: re-read S's second half from TMEM for the exponentials (0: hold all of S)
+#define SSKIP_PF_RELOAD 0     // 1, d = 128: re-read S's second half from TMEM for the exponentials (0: hold all of S)
 #endif
 #ifndef SSKIP_PF_RELOAD_D64
 #define SSKIP_PF_RELOAD_D64 0  // at d = 64 S stays in registers from the max pass
