@@ -560,15 +560,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (key >= p.L || (CAUSAL && key > row)) s[c] = -INFINITY;
         }
       }
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+      // Three-input max tree: a first level of independent maxima over column
+      // triples, then levels of three until one value is left.
+      float t[(BC + 2) / 3];
 #pragma unroll
-      for (int c = 0; c < BC; c += 8) {
-        mx0 = fmax3(mx0, s[c], s[c + 1]);
-        mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
-        mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
-        mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
+      for (int i = 0; i < BC / 3; ++i) t[i] = fmax3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
+      int n = BC / 3;
+      if (BC % 3 == 1) t[n++] = s[BC - 1];
+      if (BC % 3 == 2) t[n++] = fmaxf(s[BC - 2], s[BC - 1]);
+#pragma unroll
+      for (int level = 0; level < 5; ++level) {
+        int m = 0;
+#pragma unroll
+        for (int i = 0; i + 2 < n; i += 3) t[m++] = fmax3(t[i], t[i + 1], t[i + 2]);
+        if (n % 3 == 1) t[m++] = t[n - 1];
+        if (n % 3 == 2) t[m++] = fmaxf(t[n - 2], t[n - 1]);
+        n = m;
       }
-      const float m_loc = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * scale;  // scale > 0
+      const float m_loc = t[0] * scale;  // scale > 0
       const bool gvis = j <= my_jmax;
       const bool pass = row_passes_log2(m_loc, m_run, log2_t, t_pos);
       const bool wall = __all_sync(0xffffffffu, !(row_in && gvis) || pass);
